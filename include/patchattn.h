@@ -1,0 +1,158 @@
+/*
+ * patchattn.h -- C ABI of the B200 (sm_100a) PipeFusion patch-attention library.
+ *
+ * The library runs, on one GPU, the data path of PipeFusion's patch-level attention
+ * ("기술 요약: PipeFusion", 핵심 메커니즘 1-4; "PipeFusion: Patch-level Pipeline Parallelism
+ * for Diffusion Transformers Inference", Résumé Technique / Mécanismes Principaux):
+ *
+ *   - the image tokens of a diffusion step are cut into M non-overlapping patches, here
+ *     the contiguous row-major token ranges [p*P, (p+1)*P), P = n_img / M;
+ *   - each layer keeps a full-spatial K/V buffer; when patch p of step s is computed,
+ *     the buffer rows of patches < p already hold step s (written by the calls for those
+ *     patches), the rows of patches > p still hold step s-1 ("stale" activations of the
+ *     previous sampler step, 2. 시간적 중복성 활용), and patch p's own rows are
+ *     overwritten with the fresh K/V passed to the call;
+ *   - the patch's queries then attend to every buffer row plus the step's always-fresh
+ *     text tokens (MM-DiT joint attention), softmax(scale * Q K^T) V.
+ *
+ * and the guidance combine that feeds hybrid-CFG switching ("조건부 가이드 스케줄링 기반
+ * 하이브리드 데이터-파이프라인 병렬 처리를 통한 디퓨전 모델 가속화", second block 단락 1-3):
+ *   out = eps_u + w * (eps_c - eps_u),  rel-MAE_t = ||eps_c - eps_u||_1 / ||eps_u||_1.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - Memory: the caller owns all device memory (inputs, outputs, K/V buffers, workspace);
+ *    the library allocates no device memory.  A pf_ctx holds host state only.
+ *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Work is enqueued asynchronously; pointers must stay valid until the
+ *    stream has executed it.
+ *  - Layout: every attention tensor is contiguous row-major [batch, tokens, heads,
+ *    head_dim] bf16 (the natural output of a QKV projection); strides are derived.
+ *    All device pointers must be 16-byte aligned (else PF_ERR_ALIGN).
+ *  - Errors: every call returns pf_status; nothing aborts and no exception crosses the
+ *    ABI.  Argument, shape, order and state errors are detected on the host before any
+ *    work is enqueued, and leave the context unchanged.  Launch failures return
+ *    PF_ERR_CUDA.  Faults of enqueued work surface at the caller's next stream sync.
+ *  - Thread safety: a pf_ctx must not be used from two host threads at once.
+ */
+#ifndef PATCHATTN_H_
+#define PATCHATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PF_OK = 0,
+  PF_ERR_INVALID_ARG = 1, /* NULL where a pointer is required, negative size, bad layer/patch */
+  PF_ERR_SHAPE = 2,       /* n_img not a multiple of n_patches, zero-sized dimension */
+  PF_ERR_ALIGN = 3,       /* a device pointer is not 16-byte aligned */
+  PF_ERR_UNSUPPORTED = 4, /* head_dim not in {64, 72, 128}, unknown schedule, no sm_100 device */
+  PF_ERR_ORDER = 5,       /* patch called out of order for the layer's schedule */
+  PF_ERR_STATE = 6,       /* step before pf_kvbuf_init of that layer */
+  PF_ERR_CUDA = 7,        /* a CUDA runtime/driver call or a kernel launch failed */
+  PF_ERR_TIMEOUT = 8      /* a kernel's bounded wait expired (reported by pf_check_device_status) */
+} pf_status;
+
+/* Which rows of the other patches a patch sees.
+ *  PF_SCHED_PIPEFUSION: this step's rows for patches < p (written by the earlier calls of
+ *    the step), stale rows for patches > p.  Patches must be called 0, 1, ..., M-1 per
+ *    step, then wrap to 0 for the next step.
+ *  PF_SCHED_DISTRIFUSION: every other patch is seen at the previous step (the buffer is
+ *    only written after the last patch of the step), the schedule of DistriFusion
+ *    ("기술 요약: PipeFusion", 문제 정의: DistriFusion keeps full-spatial stale K/V).
+ *    Patches may come in any order, each once per step; the step ends after M calls. */
+typedef enum { PF_SCHED_PIPEFUSION = 0, PF_SCHED_DISTRIFUSION = 1 } pf_schedule;
+
+typedef struct {
+  int batch;           /* B >= 1 */
+  int heads;           /* H >= 1 */
+  int head_dim;        /* d in {64, 72, 128} */
+  int n_img;           /* image tokens N >= 1, multiple of n_patches */
+  int n_patches;       /* M >= 1 */
+  int n_txt;           /* text tokens T >= 0 */
+  int n_layers;        /* L >= 1: one K/V buffer per layer */
+  float softmax_scale; /* 0 => 1/sqrt(head_dim) with the real head_dim */
+  int schedule;        /* pf_schedule */
+} pf_config;
+
+typedef struct pf_ctx pf_ctx; /* opaque, host-only */
+
+/* Bytes of ONE layer's K/V buffer: K region [B, N, H, d] bf16 followed by the V region of
+ * the same size (2 * B * N * H * d * 2 bytes).  0 if cfg is NULL or invalid. */
+size_t pf_kvbuf_bytes(const pf_config* cfg);
+
+/* Create a context.  kvbuf_per_layer: host array of n_layers device pointers, each to a
+ * caller-owned buffer of pf_kvbuf_bytes(cfg) bytes that must outlive the context.
+ * On success *out receives the context; on failure *out is set to NULL. */
+pf_status pf_create(const pf_config* cfg, void* const* kvbuf_per_layer, pf_ctx** out);
+
+/* Free the host state of ctx (not the caller's buffers).  NULL => PF_OK. */
+pf_status pf_destroy(pf_ctx* ctx);
+
+/* Start-up pass ("기술 요약: PipeFusion", 핵심 메커니즘 2: stale data exists only after the
+ * initial start): copy the first step's full-spatial K and V, [B, N, H, d] bf16 each,
+ * into layer `layer`'s buffer and reset that layer's patch counter to 0.  A bit copy. */
+pf_status pf_kvbuf_init(pf_ctx* ctx, int layer, const void* k_full, const void* v_full,
+                        void* stream);
+
+/* One micro-step: layer `layer`, patch `patch` of the current step.
+ *   q_p, k_p, v_p : fresh activations of the patch, [B, P, H, d] bf16
+ *   k_txt, v_txt  : this step's text keys/values, [B, T, H, d] bf16 (both NULL iff T == 0)
+ *   o_p           : output, [B, P, H, d] bf16, o_p = softmax(scale Q_p [K';K_txt]^T) [V';V_txt]
+ *                   where K', V' is the buffer with patch p's rows replaced by k_p, v_p.
+ * Under PF_SCHED_PIPEFUSION the call also writes k_p, v_p into the buffer rows of patch p
+ * (fused into the attention kernel); o_p must not alias any input.
+ * Errors: PF_ERR_STATE before pf_kvbuf_init(layer); PF_ERR_ORDER if `patch` is not the
+ * layer's next patch; PF_ERR_INVALID_ARG / PF_ERR_ALIGN for bad pointers. */
+pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
+                             const void* k_p, const void* v_p, const void* k_txt,
+                             const void* v_txt, void* o_p, void* stream);
+
+/* Next patch index the layer expects (0 at the start of a step).  Checkpoint helper: a
+ * layer's whole state is its buffer contents plus this counter. */
+pf_status pf_get_state(const pf_ctx* ctx, int layer, int* next_patch);
+
+/* Restore a counter saved with pf_get_state (the caller restores the buffer contents). */
+pf_status pf_set_state(pf_ctx* ctx, int layer, int next_patch);
+
+/* Workspace bytes pf_cfg_combine_relmae needs for `batch` samples of `n_per_sample`
+ * floats (0 on invalid sizes). */
+size_t pf_cfg_workspace_bytes(int batch, int64_t n_per_sample);
+
+/* Guidance combine + rel-MAE_t, fused in one pass over eps_c and eps_u.
+ *   eps_c, eps_u : device fp32 [batch, n_per_sample] (any [B, C, H, W] flattened per sample)
+ *   w            : guidance weight
+ *   out_f32      : device fp32 [batch, n_per_sample] = eps_u + w (eps_c - eps_u), or NULL
+ *   out_bf16     : device bf16 (uint16 bits) same shape, round-to-nearest-even of the fp32
+ *                  result, or NULL
+ *   relmae       : device fp32 [batch]: per-sample ||eps_c - eps_u||_1 / ||eps_u||_1
+ *                  (0 if both norms are 0, +inf if only the denominator is 0)
+ *   workspace    : device scratch of pf_cfg_workspace_bytes(batch, n_per_sample) bytes,
+ *                  no initialisation needed; one workspace per concurrently running call
+ * The reduction is deterministic (fixed order, no float atomics): equal inputs give
+ * bitwise-equal outputs.  n_per_sample must be a multiple of 4 (16-byte rows). */
+pf_status pf_cfg_combine_relmae(const float* eps_c, const float* eps_u, int batch,
+                                int64_t n_per_sample, float w, float* out_f32,
+                                uint16_t* out_bf16, float* relmae, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, then read the device status word the context's kernels write when
+ * a bounded wait expires: PF_ERR_TIMEOUT if any did (and clear it), PF_ERR_CUDA if the
+ * stream reported an error, else PF_OK. */
+pf_status pf_check_device_status(pf_ctx* ctx, void* stream);
+
+/* Static description of a status code (never NULL). */
+const char* pf_status_string(pf_status s);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int pf_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PATCHATTN_H_ */

@@ -29,7 +29,9 @@ import numpy as np
 
 def softmax_probs(q: np.ndarray, k: np.ndarray, scale: float) -> np.ndarray:
     """Row-stochastic attention weights, [H, n_q, n_k], max-subtracted softmax in fp64."""
-    logits = np.einsum("qhd,khd->hqk", q, k) * scale
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    logits = np.matmul(q.transpose(1, 0, 2), k.transpose(1, 2, 0)) * scale
     logits = logits - logits.max(axis=-1, keepdims=True)
     w = np.exp(logits)
     return w / w.sum(axis=-1, keepdims=True)
@@ -38,7 +40,8 @@ def softmax_probs(q: np.ndarray, k: np.ndarray, scale: float) -> np.ndarray:
 def attend(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.ndarray:
     """O = softmax(scale * Q K^T) V per head.  q [n_q,H,d], k/v [n_k,H,d] -> [n_q,H,d]."""
     w = softmax_probs(q, k, scale)
-    return np.einsum("hqk,khd->qhd", w, v)
+    v = np.asarray(v, dtype=np.float64)
+    return np.matmul(w, v.transpose(1, 0, 2)).transpose(1, 0, 2)
 
 
 def image_key_rows(x_now: np.ndarray, x_prev: np.ndarray, p: int, n_patches: int) -> np.ndarray:

@@ -1,0 +1,478 @@
+// attn_fwd.cu -- fused KV-buffer scatter + patch attention for sm_100a (B200).
+//
+// One launch runs one PipeFusion micro-step ("기술 요약: PipeFusion", 핵심 메커니즘 1-3):
+// the queries of patch p attend to the layer's full-spatial K/V context, in which patch
+// p's own rows are the fresh K_p/V_p of the call, the other image rows come from the
+// layer buffer (this step's rows for earlier patches, the previous step's for later
+// ones), and the step's text tokens are appended (joint attention).  The same launch
+// writes K_p/V_p into the buffer rows of patch p for the calls that follow.
+//
+// Design (per CTA = one head of one batch element, NQ x 128 query rows):
+//   warps 0-3 / 4-7  softmax for query tile 0 / 1: one thread owns one query row (one
+//                    TMEM lane), so the row max and row sum need no shuffles.
+//   warp 8           TMEM allocation and the single-thread tcgen05.mma issuer.
+//   warp 9           TMA producer: Q tiles once, then K/V tiles through a smem ring.
+//   warp 10          scatter of the CTA's share of K_p/V_p into the buffer.
+// S = Q K^T lands in TMEM (fp32, 128 columns per query tile); the softmax overwrites its
+// first 64 columns with P as packed bf16, which the PV MMA reads straight from TMEM
+// (A operand in TMEM, V as an MN-major B operand in smem).  O accumulates in TMEM.
+// The context is walked as segments so that patch p's rows are read from the fresh
+// tensors, never from buffer rows that other CTAs of this launch are writing:
+//   [fresh rows 0..P) | buffer rows 0..pP) | buffer rows (p+1)P..N) | text rows 0..T)
+// Softmax is permutation invariant over keys, so this order gives the same result as
+// the natural token order.  Row maxima are kept lazily: O is rescaled only when a row's
+// maximum grows by more than 2^8, which is exact because the final O / l uses the same
+// reference maximum for numerator and denominator.
+//
+// Every wait is bounded (2 s); on expiry the kernel records the role in a device word,
+// raises a CTA-wide abort flag, drains its in-flight copies and MMAs, frees TMEM and
+// returns.
+
+#include <cuda_bf16.h>
+
+#include "pf_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace pf {
+
+__device__ unsigned int g_watchdog = 0;
+
+namespace {
+
+using namespace ptx;
+
+constexpr int kRows = 128;             // query rows per Q tile == key rows per K/V tile
+constexpr int kChunkBytes = 128 * 128; // 128 rows x 64 bf16 columns (one 128-byte swizzle span)
+constexpr int kThreads = 352;          // 11 warps
+constexpr int kWarpMma = 8;
+constexpr int kWarpLoad = 9;
+constexpr int kWarpScatter = 10;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 256;        // O_t at column 256 + 128 t; S_t at column 128 t
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+enum : unsigned { kWdLoad = 1u, kWdMma = 2u, kWdSoftmax = 4u, kWdEpilogue = 8u };
+
+template <int D>
+struct Dims {
+  static constexpr int kChunks = (D + 63) / 64;          // 64-column chunks per row
+  static constexpr int kMmaN = (D + 15) / 16 * 16;       // head_dim padded to 16 (72 -> 80)
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kStages = D <= 64 ? 8 : 4;
+};
+
+template <int D, int NQ>
+constexpr int smem_bytes() {
+  return 1024 + (NQ + Dims<D>::kStages) * Dims<D>::kTileBytes + 256;
+}
+
+// Which tensor and rows the j-th 128-row context tile comes from.
+struct Segments {
+  int n_fresh, n_lo, n_hi, n_txt;  // tiles per segment
+  int plen, lo_len, hi_row0, hi_len, txt_len;
+
+  __device__ void init(const AttnParams& p) {
+    plen = p.plen;
+    lo_len = p.patch * p.plen;
+    hi_row0 = (p.patch + 1) * p.plen;
+    hi_len = p.n_img - hi_row0;
+    txt_len = p.n_txt;
+    n_fresh = (plen + kRows - 1) / kRows;
+    n_lo = (lo_len + kRows - 1) / kRows;
+    n_hi = (hi_len + kRows - 1) / kRows;
+    n_txt = (txt_len + kRows - 1) / kRows;
+  }
+  __device__ int total() const { return n_fresh + n_lo + n_hi + n_txt; }
+  // src: 0 = fresh tensors, 1 = buffer, 2 = text
+  __device__ void tile(int j, int& src, int& row0, int& nvalid) const {
+    if (j < n_fresh) {
+      src = 0; row0 = j * kRows; nvalid = min(kRows, plen - row0); return;
+    }
+    j -= n_fresh;
+    if (j < n_lo) {
+      src = 1; row0 = j * kRows; nvalid = min(kRows, lo_len - row0); return;
+    }
+    j -= n_lo;
+    if (j < n_hi) {
+      src = 1; row0 = hi_row0 + j * kRows; nvalid = min(kRows, hi_len - j * kRows); return;
+    }
+    j -= n_hi;
+    src = 2; row0 = j * kRows; nvalid = min(kRows, txt_len - row0);
+  }
+  __device__ int nvalid(int j) const {
+    int s, r, n;
+    tile(j, s, r, n);
+    return n;
+  }
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void raise_abort(volatile int* abort, unsigned code) {
+  *abort = 1;
+  atomicOr(&g_watchdog, code);
+}
+
+template <int D, int NQ>
+__global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_constant__ AttnParams p) {
+  using Dm = Dims<D>;
+  constexpr int S = Dm::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + NQ * Dm::kTileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + S * Dm::kTileBytes);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + S;
+  uint64_t* s_full = kv_empty + S;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_full = p_full + 2;
+  uint64_t* mma_done = o_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int q0 = blockIdx.x * NQ * kRows;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(q_full), 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(kv_full + s), 1);
+      mbar_init(smem_u32(kv_empty + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(smem_u32(s_full + t), 1);
+      mbar_init(smem_u32(p_full + t), kRows);
+      mbar_init(smem_u32(o_full + t), 1);
+    }
+    mbar_init(smem_u32(mma_done), 1);
+    *abort = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kWarpLoad && lane == 0) {
+    prefetch_tmap(&p.tm_q);
+    prefetch_tmap(&p.tm_kf);
+    prefetch_tmap(&p.tm_vf);
+    prefetch_tmap(&p.tm_kb);
+    prefetch_tmap(&p.tm_vb);
+    if (p.n_txt > 0) {
+      prefetch_tmap(&p.tm_kt);
+      prefetch_tmap(&p.tm_vt);
+    }
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  Segments seg;
+  seg.init(p);
+  const int n_tiles = seg.total();
+
+  if (warp == kWarpLoad) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint32_t qbar = smem_u32(q_full);
+      mbar_arrive_expect_tx(qbar, NQ * Dm::kTileBytes);
+      for (int t = 0; t < NQ; ++t)
+        for (int c = 0; c < Dm::kChunks; ++c)
+          tma_load_4d(smem_u32(sQ + t * Dm::kTileBytes + c * kChunkBytes), &p.tm_q, c * 64, h,
+                      q0 + t * kRows, b, qbar);
+      int issued = 0;
+      bool ok = true;
+      for (int j = 0; j < n_tiles && ok; ++j) {
+        int src, row0, nv;
+        seg.tile(j, src, row0, nv);
+        for (int kv = 0; kv < 2; ++kv) {
+          const int i = 2 * j + kv;
+          const int st = i % S;
+          if (!mbar_wait(smem_u32(kv_empty + st), ((i / S) & 1) ^ 1, abort, kWaitNs)) {
+            ok = false;
+            break;
+          }
+          const CUtensorMap* m = src == 0 ? (kv ? &p.tm_vf : &p.tm_kf)
+                                 : src == 1 ? (kv ? &p.tm_vb : &p.tm_kb)
+                                            : (kv ? &p.tm_vt : &p.tm_kt);
+          const uint32_t fb = smem_u32(kv_full + st);
+          mbar_arrive_expect_tx(fb, Dm::kTileBytes);
+          for (int c = 0; c < Dm::kChunks; ++c)
+            tma_load_4d(smem_u32(sKV + st * Dm::kTileBytes + c * kChunkBytes), m, c * 64, h, row0,
+                        b, fb);
+          issued = i + 1;
+        }
+      }
+      if (!ok) raise_abort(abort, kWdLoad);
+      // drain: every issued copy must land before the CTA exits
+      mbar_wait(qbar, 0, nullptr, kWaitNs);
+      for (int i = issued > S ? issued - S : 0; i < issued; ++i)
+        mbar_wait(smem_u32(kv_full + (i % S)), (i / S) & 1, nullptr, kWaitNs);
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, Dm::kMmaN, 1);
+      const uint32_t q_base = smem_u32(sQ);
+      const uint32_t kv_base = smem_u32(sKV);
+
+      auto issue_qk = [&](int t, int st) {
+        const uint32_t a0 = q_base + t * Dm::kTileBytes;
+        const uint32_t b0 = kv_base + st * Dm::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < Dm::kMmaN / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
+          mma_ss(tmem + t * 128, smem_desc_sw128(a0 + off, 16, 1024),
+                 smem_desc_sw128(b0 + off, 16, 1024), idesc_qk, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int t, int st, bool acc) {
+        const uint32_t v0 = kv_base + st * Dm::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk) {
+          mma_ts(tmem + kColO + t * 128, tmem + t * 128 + kk * 8,
+                 smem_desc_sw128(v0 + kk * 2048, kChunkBytes, 1024), idesc_pv, acc || kk > 0);
+        }
+      };
+
+      bool ok = mbar_wait(smem_u32(q_full), 0, abort, kWaitNs);
+      tc_fence_after();
+      for (int j = 0; j < n_tiles && ok; ++j) {
+        const int iK = 2 * j, sK = iK % S;
+        if (!(ok = mbar_wait(smem_u32(kv_full + sK), (iK / S) & 1, abort, kWaitNs))) break;
+        tc_fence_after();
+        int sV = 0;
+        if (j > 0) {
+          const int iV = 2 * j - 1;
+          sV = iV % S;
+          if (!(ok = mbar_wait(smem_u32(kv_full + sV), (iV / S) & 1, abort, kWaitNs))) break;
+          tc_fence_after();
+        }
+        for (int t = 0; t < NQ; ++t) {
+          if (j > 0) {
+            if (!(ok = mbar_wait(smem_u32(p_full + t), (j - 1) & 1, abort, kWaitNs))) break;
+            tc_fence_after();
+            issue_pv(t, sV, j - 1 > 0);
+          }
+          issue_qk(t, sK);
+          mma_commit(smem_u32(s_full + t));
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(kv_empty + sK));
+        if (j > 0) mma_commit(smem_u32(kv_empty + sV));
+      }
+      if (ok && n_tiles > 0) {
+        const int iV = 2 * n_tiles - 1, sV = iV % S;
+        ok = mbar_wait(smem_u32(kv_full + sV), (iV / S) & 1, abort, kWaitNs);
+        tc_fence_after();
+        for (int t = 0; t < NQ && ok; ++t) {
+          if (!(ok = mbar_wait(smem_u32(p_full + t), (n_tiles - 1) & 1, abort, kWaitNs))) break;
+          tc_fence_after();
+          issue_pv(t, sV, n_tiles - 1 > 0);
+          mma_commit(smem_u32(o_full + t));
+        }
+        if (ok) mma_commit(smem_u32(kv_empty + sV));
+      }
+      if (!ok) raise_abort(abort, kWdMma);
+      // drain every MMA issued by this thread before TMEM is released
+      mma_commit(smem_u32(mma_done));
+      mbar_wait(smem_u32(mma_done), 0, nullptr, kWaitNs);
+    }
+  } else if (warp == kWarpScatter) {
+    // ------------------------------------------------------------ buffer scatter
+    if (p.k_dst != nullptr) {
+      constexpr int kVec = D / 8;  // 16-byte vectors per row of one head
+      const int r0 = q0;
+      const int r1 = min(q0 + NQ * kRows, p.plen);
+      const int total = (r1 - r0) * kVec;
+      const size_t src_row_stride = static_cast<size_t>(p.heads) * D;
+      const size_t dst_row0 = static_cast<size_t>(b) * p.n_img + static_cast<size_t>(p.patch) * p.plen;
+      const uint4* ksrc = reinterpret_cast<const uint4*>(p.k_p);
+      const uint4* vsrc = reinterpret_cast<const uint4*>(p.v_p);
+      uint4* kdst = reinterpret_cast<uint4*>(p.k_dst);
+      uint4* vdst = reinterpret_cast<uint4*>(p.v_dst);
+      for (int base = lane; base < total; base += 32 * 4) {
+        uint4 kx[4], vx[4];
+        size_t so[4], dof[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = base + u * 32;
+          if (i < total) {
+            const int r = r0 + i / kVec, v = i % kVec;
+            so[u] = ((static_cast<size_t>(b) * p.plen + r) * src_row_stride + static_cast<size_t>(h) * D) / 8 + v;
+            dof[u] = ((dst_row0 + r) * src_row_stride + static_cast<size_t>(h) * D) / 8 + v;
+            kx[u] = __ldg(ksrc + so[u]);
+            vx[u] = __ldg(vsrc + so[u]);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (base + u * 32 < total) {
+            kdst[dof[u]] = kx[u];
+            vdst[dof[u]] = vx[u];
+          }
+        }
+      }
+    }
+  } else if (warp < 4 * NQ) {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int t = warp >> 2;
+    const int wq = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + kColO + t * 128;
+    const float c = p.scale_log2;
+    float m = -INFINITY;  // reference row maximum, already scaled to log2 units
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      ok = mbar_wait(smem_u32(s_full + t), j & 1, abort, kWaitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[128];
+      tmem_ld32(tS + 0, s);
+      tmem_ld32(tS + 32, s + 32);
+      tmem_ld32(tS + 64, s + 64);
+      tmem_ld32(tS + 96, s + 96);
+      tmem_wait_ld();
+      reg_fence<128>(s);
+      const int nv = seg.nvalid(j);
+      if (nv < kRows) {
+#pragma unroll
+        for (int k = 0; k < 128; ++k)
+          if (k >= nv) s[k] = __float_as_uint(-INFINITY);
+      }
+      float mx = __uint_as_float(s[0]);
+#pragma unroll
+      for (int k = 1; k < 128; ++k) mx = fmaxf(mx, __uint_as_float(s[k]));
+      const float mxs = mx * c;
+      if (mxs > m + 8.f) {
+        const float alpha = ex2(m - mxs);
+        l *= alpha;
+        if (j > 0) {
+#pragma unroll
+          for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
+            uint32_t o[16];
+            tmem_ld16(tO + c0, o);
+            tmem_wait_ld();
+            reg_fence<16>(o);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st16(tO + c0, o);
+          }
+        }
+        m = mxs;
+      }
+      const float nm = -m;
+      uint32_t pk[64];
+#pragma unroll
+      for (int k = 0; k < 64; ++k) {
+        const float p0 = ex2(fmaf(__uint_as_float(s[2 * k]), c, nm));
+        const float p1 = ex2(fmaf(__uint_as_float(s[2 * k + 1]), c, nm));
+        l += p0 + p1;
+        pk[k] = pack_bf16(p0, p1);
+      }
+      tmem_st32(tS, pk);
+      tmem_st32(tS + 32, pk + 32);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(p_full + t));
+    }
+    if (!ok) {
+      if (lane == 0) raise_abort(abort, kWdSoftmax);
+    } else {
+      ok = mbar_wait(smem_u32(o_full + t), 0, abort, kWaitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) raise_abort(abort, kWdEpilogue);
+      } else {
+        tc_fence_after();
+        const int row = q0 + t * kRows + wq * 32 + lane;
+        const float inv = 1.f / l;
+        uint16_t* dst = p.o + ((static_cast<size_t>(b) * p.plen + row) * p.heads + h) * D;
+        const bool in_range = row < p.plen;
+#pragma unroll
+        for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
+          uint32_t o[16];
+          tmem_ld16(tO + c0, o);
+          tmem_wait_ld();
+          reg_fence<16>(o);
+          uint4 w0, w1;
+          w0.x = pack_bf16(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);
+          w0.y = pack_bf16(__uint_as_float(o[2]) * inv, __uint_as_float(o[3]) * inv);
+          w0.z = pack_bf16(__uint_as_float(o[4]) * inv, __uint_as_float(o[5]) * inv);
+          w0.w = pack_bf16(__uint_as_float(o[6]) * inv, __uint_as_float(o[7]) * inv);
+          w1.x = pack_bf16(__uint_as_float(o[8]) * inv, __uint_as_float(o[9]) * inv);
+          w1.y = pack_bf16(__uint_as_float(o[10]) * inv, __uint_as_float(o[11]) * inv);
+          w1.z = pack_bf16(__uint_as_float(o[12]) * inv, __uint_as_float(o[13]) * inv);
+          w1.w = pack_bf16(__uint_as_float(o[14]) * inv, __uint_as_float(o[15]) * inv);
+          if (in_range) {
+            if (c0 + 8 <= D) *reinterpret_cast<uint4*>(dst + c0) = w0;
+            if (c0 + 16 <= D) *reinterpret_cast<uint4*>(dst + c0 + 8) = w1;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D, int NQ>
+cudaError_t launch_one(const AttnParams& p, cudaStream_t stream) {
+  constexpr int smem = smem_bytes<D, NQ>();
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(patch_attn_kernel<D, NQ>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  dim3 grid((p.plen + NQ * kRows - 1) / (NQ * kRows), p.heads, p.batch);
+  patch_attn_kernel<D, NQ><<<grid, kThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_patch_attn(const AttnParams& p, cudaStream_t stream) {
+  const bool two = p.plen > kRows;
+  switch (p.head_dim) {
+    case 64: return two ? launch_one<64, 2>(p, stream) : launch_one<64, 1>(p, stream);
+    case 72: return two ? launch_one<72, 2>(p, stream) : launch_one<72, 1>(p, stream);
+    case 128: return two ? launch_one<128, 2>(p, stream) : launch_one<128, 1>(p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t read_and_clear_watchdog(unsigned* value) {
+  unsigned v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_watchdog, sizeof(v));
+  if (e != cudaSuccess) return e;
+  *value = v;
+  if (v != 0) {
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_watchdog, &zero, sizeof(zero));
+  }
+  return e;
+}
+
+}  // namespace pf

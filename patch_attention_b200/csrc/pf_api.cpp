@@ -1,0 +1,297 @@
+// pf_api.cpp -- host side of the C ABI declared in include/patchattn.h.
+//
+// Validates every argument before anything is enqueued, keeps the per-layer schedule
+// state (which patch comes next, which buffer half is read), encodes the TMA tensor maps
+// of each micro-step and launches the kernels.  Holds no device memory.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "patchattn.h"
+#include "pf_internal.h"
+
+struct pf_ctx {
+  pf_config cfg;
+  float scale;
+  size_t tensor_elems;           // B * N * H * d: one K or V region of a buffer
+  std::vector<uint8_t*> base;    // per layer, caller-owned
+  std::vector<int> next_patch;   // PipeFusion: the patch the layer expects next
+  std::vector<int> initialised;
+  std::vector<int> read_half;    // DistriFusion: which half of the buffer holds the stale step
+  std::vector<std::vector<uint8_t>> seen;  // DistriFusion: patches done in the current step
+  std::vector<int> seen_count;
+};
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool config_ok(const pf_config* c) {
+  return c && c->batch >= 1 && c->heads >= 1 && c->n_img >= 1 && c->n_patches >= 1 &&
+         c->n_txt >= 0 && c->n_layers >= 1;
+}
+
+pf_status check_config(const pf_config* c) {
+  if (!c) return PF_ERR_INVALID_ARG;
+  if (c->batch < 1 || c->heads < 1 || c->n_img < 1 || c->n_patches < 1 || c->n_txt < 0 ||
+      c->n_layers < 1)
+    return PF_ERR_SHAPE;
+  if (c->n_img % c->n_patches != 0) return PF_ERR_SHAPE;
+  if (c->head_dim != 64 && c->head_dim != 72 && c->head_dim != 128) return PF_ERR_UNSUPPORTED;
+  if (c->schedule != PF_SCHED_PIPEFUSION && c->schedule != PF_SCHED_DISTRIFUSION)
+    return PF_ERR_UNSUPPORTED;
+  if (!(c->softmax_scale >= 0.f) || std::isinf(c->softmax_scale)) return PF_ERR_INVALID_ARG;
+  // TMA coordinates and per-row offsets are 32-bit
+  const double rows = static_cast<double>(c->batch) * c->n_img;
+  if (rows > 2e9 || static_cast<double>(c->n_txt) * c->batch > 2e9) return PF_ERR_SHAPE;
+  return PF_OK;
+}
+
+size_t region_elems(const pf_config* c) {
+  return static_cast<size_t>(c->batch) * c->n_img * c->heads * c->head_dim;
+}
+
+// [batch, rows, heads, d] bf16 -> 4-D tensor map, box = 64 columns x 1 head x 128 rows.
+bool make_map(CUtensorMap* m, const void* base, int batch, int rows, int heads, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(batch)};
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(heads) * d * 2;
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, row_bytes,
+                                 row_bytes * static_cast<cuuint64_t>(rows)};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+pf_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PF_OK : PF_ERR_CUDA; }
+
+bool layer_ok(const pf_ctx* ctx, int layer) { return layer >= 0 && layer < ctx->cfg.n_layers; }
+
+// K/V regions of a layer's buffer: half 0 is [K | V]; DistriFusion adds half 1 [K | V].
+uint8_t* region(const pf_ctx* ctx, int layer, int half, int kv) {
+  const size_t bytes = ctx->tensor_elems * 2;
+  return ctx->base[layer] + (static_cast<size_t>(half) * 2 + kv) * bytes;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t pf_kvbuf_bytes(const pf_config* cfg) {
+  if (check_config(cfg) != PF_OK) return 0;
+  const size_t halves = cfg->schedule == PF_SCHED_DISTRIFUSION ? 2 : 1;
+  return halves * 2 * region_elems(cfg) * 2;
+}
+
+pf_status pf_create(const pf_config* cfg, void* const* kvbuf_per_layer, pf_ctx** out) {
+  if (!out) return PF_ERR_INVALID_ARG;
+  *out = nullptr;
+  pf_status st = check_config(cfg);
+  if (st != PF_OK) return st;
+  if (!kvbuf_per_layer) return PF_ERR_INVALID_ARG;
+  for (int l = 0; l < cfg->n_layers; ++l) {
+    if (!kvbuf_per_layer[l]) return PF_ERR_INVALID_ARG;
+    if (!aligned16(kvbuf_per_layer[l])) return PF_ERR_ALIGN;
+  }
+  pf_ctx* ctx = new (std::nothrow) pf_ctx();
+  if (!ctx) return PF_ERR_INVALID_ARG;
+  ctx->cfg = *cfg;
+  ctx->scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale
+                                        : 1.0f / std::sqrt(static_cast<float>(cfg->head_dim));
+  ctx->tensor_elems = region_elems(cfg);
+  ctx->base.resize(cfg->n_layers);
+  for (int l = 0; l < cfg->n_layers; ++l) ctx->base[l] = static_cast<uint8_t*>(kvbuf_per_layer[l]);
+  ctx->next_patch.assign(cfg->n_layers, 0);
+  ctx->initialised.assign(cfg->n_layers, 0);
+  ctx->read_half.assign(cfg->n_layers, 0);
+  ctx->seen.assign(cfg->n_layers, std::vector<uint8_t>(cfg->n_patches, 0));
+  ctx->seen_count.assign(cfg->n_layers, 0);
+  *out = ctx;
+  return PF_OK;
+}
+
+pf_status pf_destroy(pf_ctx* ctx) {
+  delete ctx;
+  return PF_OK;
+}
+
+pf_status pf_kvbuf_init(pf_ctx* ctx, int layer, const void* k_full, const void* v_full,
+                        void* stream) {
+  if (!ctx || !k_full || !v_full) return PF_ERR_INVALID_ARG;
+  if (!layer_ok(ctx, layer)) return PF_ERR_INVALID_ARG;
+  if (!aligned16(k_full) || !aligned16(v_full)) return PF_ERR_ALIGN;
+  const int half = ctx->read_half[layer];
+  cudaError_t e = pf::launch_kvbuf_copy(k_full, v_full, region(ctx, layer, half, 0),
+                                        region(ctx, layer, half, 1), ctx->tensor_elems,
+                                        static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return PF_ERR_CUDA;
+  ctx->initialised[layer] = 1;
+  ctx->next_patch[layer] = 0;
+  std::fill(ctx->seen[layer].begin(), ctx->seen[layer].end(), 0);
+  ctx->seen_count[layer] = 0;
+  return PF_OK;
+}
+
+pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
+                             const void* k_p, const void* v_p, const void* k_txt,
+                             const void* v_txt, void* o_p, void* stream) {
+  if (!ctx) return PF_ERR_INVALID_ARG;
+  const pf_config& c = ctx->cfg;
+  if (!layer_ok(ctx, layer) || patch < 0 || patch >= c.n_patches) return PF_ERR_INVALID_ARG;
+  if (!q_p || !k_p || !v_p || !o_p) return PF_ERR_INVALID_ARG;
+  if (c.n_txt > 0 && (!k_txt || !v_txt)) return PF_ERR_INVALID_ARG;
+  if (c.n_txt == 0 && (k_txt || v_txt)) return PF_ERR_INVALID_ARG;
+  if (!aligned16(q_p) || !aligned16(k_p) || !aligned16(v_p) || !aligned16(o_p) ||
+      (k_txt && !aligned16(k_txt)) || (v_txt && !aligned16(v_txt)))
+    return PF_ERR_ALIGN;
+  if (!ctx->initialised[layer]) return PF_ERR_STATE;
+  const bool pipefusion = c.schedule == PF_SCHED_PIPEFUSION;
+  if (pipefusion) {
+    if (patch != ctx->next_patch[layer]) return PF_ERR_ORDER;
+  } else {
+    if (ctx->seen[layer][patch]) return PF_ERR_ORDER;
+  }
+
+  const int plen = c.n_img / c.n_patches;
+  const int d = c.head_dim;
+  pf::AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int read = ctx->read_half[layer];
+  const int write = pipefusion ? read : 1 - read;
+  if (!make_map(&p.tm_q, q_p, c.batch, plen, c.heads, d) ||
+      !make_map(&p.tm_kf, k_p, c.batch, plen, c.heads, d) ||
+      !make_map(&p.tm_vf, v_p, c.batch, plen, c.heads, d) ||
+      !make_map(&p.tm_kb, region(ctx, layer, read, 0), c.batch, c.n_img, c.heads, d) ||
+      !make_map(&p.tm_vb, region(ctx, layer, read, 1), c.batch, c.n_img, c.heads, d))
+    return PF_ERR_CUDA;
+  if (c.n_txt > 0 && (!make_map(&p.tm_kt, k_txt, c.batch, c.n_txt, c.heads, d) ||
+                      !make_map(&p.tm_vt, v_txt, c.batch, c.n_txt, c.heads, d)))
+    return PF_ERR_CUDA;
+  p.k_p = static_cast<const uint16_t*>(k_p);
+  p.v_p = static_cast<const uint16_t*>(v_p);
+  p.k_dst = reinterpret_cast<uint16_t*>(region(ctx, layer, write, 0));
+  p.v_dst = reinterpret_cast<uint16_t*>(region(ctx, layer, write, 1));
+  p.o = static_cast<uint16_t*>(o_p);
+  p.batch = c.batch;
+  p.heads = c.heads;
+  p.plen = plen;
+  p.n_img = c.n_img;
+  p.n_txt = c.n_txt;
+  p.patch = patch;
+  p.head_dim = d;
+  p.scale_log2 = ctx->scale * 1.4426950408889634f;
+
+  cudaError_t e = pf::launch_patch_attn(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return PF_ERR_CUDA;
+
+  if (pipefusion) {
+    ctx->next_patch[layer] = (patch + 1) % c.n_patches;
+  } else {
+    ctx->seen[layer][patch] = 1;
+    if (++ctx->seen_count[layer] == c.n_patches) {
+      // every patch of the step wrote its fresh rows into the other half: it becomes the
+      // stale context of the next step
+      ctx->read_half[layer] = 1 - ctx->read_half[layer];
+      std::fill(ctx->seen[layer].begin(), ctx->seen[layer].end(), 0);
+      ctx->seen_count[layer] = 0;
+    }
+    ctx->next_patch[layer] = ctx->seen_count[layer];
+  }
+  return PF_OK;
+}
+
+pf_status pf_get_state(const pf_ctx* ctx, int layer, int* next_patch) {
+  if (!ctx || !next_patch || !layer_ok(ctx, layer)) return PF_ERR_INVALID_ARG;
+  if (!ctx->initialised[layer]) return PF_ERR_STATE;
+  *next_patch = ctx->next_patch[layer];
+  return PF_OK;
+}
+
+pf_status pf_set_state(pf_ctx* ctx, int layer, int next_patch) {
+  if (!ctx || !layer_ok(ctx, layer)) return PF_ERR_INVALID_ARG;
+  if (next_patch < 0 || next_patch >= ctx->cfg.n_patches) return PF_ERR_INVALID_ARG;
+  if (ctx->cfg.schedule != PF_SCHED_PIPEFUSION && next_patch != 0) return PF_ERR_UNSUPPORTED;
+  ctx->next_patch[layer] = next_patch;
+  ctx->initialised[layer] = 1;
+  return PF_OK;
+}
+
+size_t pf_cfg_workspace_bytes(int batch, int64_t n_per_sample) {
+  if (batch < 1 || n_per_sample < 4 || n_per_sample % 4 != 0) return 0;
+  return pf::cfg_workspace_bytes(batch, n_per_sample);
+}
+
+pf_status pf_cfg_combine_relmae(const float* eps_c, const float* eps_u, int batch,
+                                int64_t n_per_sample, float w, float* out_f32,
+                                uint16_t* out_bf16, float* relmae, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (!eps_c || !eps_u || !relmae || !workspace) return PF_ERR_INVALID_ARG;
+  if (batch < 1 || n_per_sample < 4) return PF_ERR_SHAPE;
+  if (n_per_sample % 4 != 0) return PF_ERR_SHAPE;
+  if (static_cast<double>(batch) * static_cast<double>(n_per_sample) > 9.0e15) return PF_ERR_SHAPE;
+  if (!std::isfinite(w)) return PF_ERR_INVALID_ARG;
+  if (!aligned16(eps_c) || !aligned16(eps_u) || (out_f32 && !aligned16(out_f32)) ||
+      (out_bf16 && (reinterpret_cast<uintptr_t>(out_bf16) & 7u)) ||
+      (reinterpret_cast<uintptr_t>(relmae) & 3u) || !aligned16(workspace))
+    return PF_ERR_ALIGN;
+  if (workspace_bytes < pf::cfg_workspace_bytes(batch, n_per_sample)) return PF_ERR_INVALID_ARG;
+  return from_cuda(pf::launch_cfg_combine_relmae(eps_c, eps_u, batch, n_per_sample, w, out_f32,
+                                                 out_bf16, relmae, workspace,
+                                                 static_cast<cudaStream_t>(stream)));
+}
+
+pf_status pf_check_device_status(pf_ctx* ctx, void* stream) {
+  if (!ctx) return PF_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PF_ERR_CUDA;
+  unsigned v = 0;
+  if (pf::read_and_clear_watchdog(&v) != cudaSuccess) return PF_ERR_CUDA;
+  return v ? PF_ERR_TIMEOUT : PF_OK;
+}
+
+const char* pf_status_string(pf_status s) {
+  switch (s) {
+    case PF_OK: return "ok";
+    case PF_ERR_INVALID_ARG: return "invalid argument";
+    case PF_ERR_SHAPE: return "invalid shape";
+    case PF_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case PF_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PF_ERR_ORDER: return "patch out of order";
+    case PF_ERR_STATE: return "layer buffer not initialised";
+    case PF_ERR_CUDA: return "CUDA error";
+    case PF_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+int pf_version(void) { return 100; }
+
+}  // extern "C"

@@ -123,7 +123,9 @@ def _stream_seed(seed: int, tensor: str, layer: int) -> int:
 
 def default_seed(name: str) -> int:
     order = ["tiny", "pixart", "sd3", "flux", "cfg"]
-    return 20260000 + order.index(name)
+    if name in order:
+        return 20260000 + order.index(name)
+    return 20261000 + sum(ord(ch) * 31 ** i for i, ch in enumerate(name)) % 100000
 
 
 # ----------------------------------------------------------------------------------------

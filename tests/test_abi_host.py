@@ -1,0 +1,166 @@
+"""C ABI checks that need no GPU: the library loads, exports every declared entry point,
+and rejects bad arguments on the host before anything is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import patch_attention_b200 as pa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "patchattn.h")
+
+FAKE = 0x7F0000000000  # 16-byte aligned fake device address, never dereferenced on these paths
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pf_[a-z0-9_]+)\s*\(", src)))
+
+
+def _cfg(**kw):
+    base = dict(batch=1, heads=2, head_dim=64, n_img=256, n_patches=4, n_txt=0, n_layers=2)
+    base.update(kw)
+    return pa.make_config(**base)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(pa.library_path())
+    declared = _declared()
+    assert set(declared) == set(pa.EXPORTED), declared
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version():
+    for s in range(0, 9):
+        assert pa.pf_status_string(s)
+    assert pa.pf_status_string(99) == "unknown status"
+    assert pa.pf_version() >= 100
+
+
+def test_kvbuf_bytes():
+    c = _cfg()
+    assert pa.pf_kvbuf_bytes(c) == 2 * 1 * 256 * 2 * 64 * 2
+    c = _cfg(schedule=pa.PF_SCHED_DISTRIFUSION)
+    assert pa.pf_kvbuf_bytes(c) == 2 * 2 * 1 * 256 * 2 * 64 * 2
+    assert pa.pf_kvbuf_bytes(_cfg(n_img=255)) == 0
+    assert pa.pf_kvbuf_bytes(_cfg(head_dim=96)) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(n_img=250), pa.PF_ERR_SHAPE),
+    (dict(head_dim=96), pa.PF_ERR_UNSUPPORTED),
+    (dict(heads=0), pa.PF_ERR_SHAPE),
+    (dict(n_txt=-1), pa.PF_ERR_SHAPE),
+    (dict(schedule=7), pa.PF_ERR_UNSUPPORTED),
+    (dict(softmax_scale=-1.0), pa.PF_ERR_INVALID_ARG),
+])
+def test_create_rejects_bad_config(kw, status):
+    with pytest.raises(pa.PatchAttnError) as e:
+        pa.pf_create(_cfg(**kw), [FAKE, FAKE])
+    assert e.value.status == status
+
+
+def test_create_rejects_bad_buffers():
+    with pytest.raises(pa.PatchAttnError) as e:
+        pa.pf_create(_cfg(), [FAKE, 0])
+    assert e.value.status == pa.PF_ERR_INVALID_ARG
+    with pytest.raises(pa.PatchAttnError) as e:
+        pa.pf_create(_cfg(), [FAKE, FAKE + 8])
+    assert e.value.status == pa.PF_ERR_ALIGN
+
+
+def _raw_step(ctx, layer, patch, ptrs, txt=(None, None)):
+    L = pa._lib()
+    q, k, v, o = ptrs
+    return L.pf_patch_attn_step(ctx, layer, patch, q, k, v, txt[0], txt[1], o, None)
+
+
+def test_step_state_and_order_checks():
+    ctx = pa.pf_create(_cfg(), [FAKE, FAKE])
+    try:
+        good = (FAKE, FAKE + 4096, FAKE + 8192, FAKE + 16384)
+        # before the start-up pass
+        assert _raw_step(ctx, 0, 0, good) == pa.PF_ERR_STATE
+        # bad layer / patch / pointers are argument errors
+        assert _raw_step(ctx, 2, 0, good) == pa.PF_ERR_INVALID_ARG
+        assert _raw_step(ctx, -1, 0, good) == pa.PF_ERR_INVALID_ARG
+        assert _raw_step(ctx, 0, 4, good) == pa.PF_ERR_INVALID_ARG
+        assert _raw_step(ctx, 0, 0, (None, FAKE, FAKE, FAKE)) == pa.PF_ERR_INVALID_ARG
+        assert _raw_step(ctx, 0, 0, (FAKE + 2, FAKE, FAKE, FAKE)) == pa.PF_ERR_ALIGN
+        # text pointers must be NULL when there is no text
+        assert _raw_step(ctx, 0, 0, good, (FAKE, FAKE)) == pa.PF_ERR_INVALID_ARG
+        # restore a checkpointed counter, then the order is enforced
+        pa.pf_set_state(ctx, 0, 2)
+        assert pa.pf_get_state(ctx, 0) == 2
+        assert _raw_step(ctx, 0, 0, good) == pa.PF_ERR_ORDER
+        assert _raw_step(ctx, 0, 3, good) == pa.PF_ERR_ORDER
+        with pytest.raises(pa.PatchAttnError):
+            pa.pf_get_state(ctx, 1)  # layer 1 never initialised
+        with pytest.raises(pa.PatchAttnError):
+            pa.pf_set_state(ctx, 0, 4)
+    finally:
+        pa.pf_destroy(ctx)
+
+
+def test_step_requires_text_when_configured():
+    ctx = pa.pf_create(_cfg(n_txt=8), [FAKE, FAKE])
+    try:
+        pa.pf_set_state(ctx, 0, 0)
+        good = (FAKE, FAKE, FAKE, FAKE)
+        assert _raw_step(ctx, 0, 0, good) == pa.PF_ERR_INVALID_ARG
+        assert _raw_step(ctx, 0, 0, good, (FAKE, None)) == pa.PF_ERR_INVALID_ARG
+        assert _raw_step(ctx, 0, 0, good, (FAKE, FAKE + 4)) == pa.PF_ERR_ALIGN
+    finally:
+        pa.pf_destroy(ctx)
+
+
+def test_failed_launch_does_not_advance_order():
+    # Without a usable device the call fails after validation; the counter must not move.
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("needs a host without a GPU")
+    ctx = pa.pf_create(_cfg(), [FAKE, FAKE])
+    try:
+        pa.pf_set_state(ctx, 0, 1)
+        st = _raw_step(ctx, 0, 1, (FAKE, FAKE, FAKE, FAKE))
+        assert st == pa.PF_ERR_CUDA
+        assert pa.pf_get_state(ctx, 0) == 1
+    finally:
+        pa.pf_destroy(ctx)
+
+
+def test_destroy_null_is_ok():
+    assert pa._lib().pf_destroy(None) == pa.PF_OK
+
+
+def test_null_context_everywhere():
+    L = pa._lib()
+    assert L.pf_kvbuf_init(None, 0, FAKE, FAKE, None) == pa.PF_ERR_INVALID_ARG
+    assert L.pf_patch_attn_step(None, 0, 0, FAKE, FAKE, FAKE, None, None, FAKE, None) == pa.PF_ERR_INVALID_ARG
+    assert L.pf_check_device_status(None, None) == pa.PF_ERR_INVALID_ARG
+    out = ctypes.c_void_p()
+    assert L.pf_create(None, None, ctypes.byref(out)) == pa.PF_ERR_INVALID_ARG
+    assert out.value is None
+
+
+def test_cfg_argument_checks():
+    L = pa._lib()
+    ws = pa.pf_cfg_workspace_bytes(2, 1024)
+    assert ws >= 2 * 16
+    assert pa.pf_cfg_workspace_bytes(2, 1022) == 0
+    call = lambda **kw: L.pf_cfg_combine_relmae(
+        kw.get("c", FAKE), kw.get("u", FAKE), kw.get("b", 2), kw.get("n", 1024), kw.get("w", 7.0),
+        kw.get("of", FAKE), kw.get("ob", None), kw.get("r", FAKE), kw.get("ws", FAKE),
+        kw.get("wsb", ws), None)
+    assert call(c=None) == pa.PF_ERR_INVALID_ARG
+    assert call(r=None) == pa.PF_ERR_INVALID_ARG
+    assert call(n=1022) == pa.PF_ERR_SHAPE
+    assert call(b=0) == pa.PF_ERR_SHAPE
+    assert call(w=float("nan")) == pa.PF_ERR_INVALID_ARG
+    assert call(u=FAKE + 4) == pa.PF_ERR_ALIGN
+    assert call(ob=FAKE + 2) == pa.PF_ERR_ALIGN
+    assert call(wsb=ws - 1) == pa.PF_ERR_INVALID_ARG
