@@ -112,6 +112,18 @@ pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
                              const void* k_p, const void* v_p, const void* k_txt,
                              const void* v_txt, void* o_p, void* stream);
 
+/* Bytes of the optional attention workspace for this configuration (0 if cfg is invalid).
+ * With a workspace set, a call may split each query tile's key range over several CTAs so
+ * that the grid fills the GPU's SMs in near-whole waves; the parts are merged exactly in
+ * the log-sum-exp sense (rescaled by their row maxima) by the last part to finish. */
+size_t pf_workspace_bytes(const pf_config* cfg);
+
+/* Attach a caller-owned device workspace (16-byte aligned, >= pf_workspace_bytes(cfg))
+ * to ctx and zero its counters on `stream`.  ws = NULL detaches it (no key-range split).
+ * Calls that share a workspace must not run concurrently (one workspace per stream).
+ * After PF_ERR_TIMEOUT, set the workspace again to re-zero the counters. */
+pf_status pf_set_workspace(pf_ctx* ctx, void* ws, size_t ws_bytes, void* stream);
+
 /* Next patch index the layer expects (0 at the start of a step).  Checkpoint helper: a
  * layer's whole state is its buffer contents plus this counter. */
 pf_status pf_get_state(const pf_ctx* ctx, int layer, int* next_patch);

@@ -34,7 +34,8 @@ PF_SCHED_DISTRIFUSION = 1
 
 EXPORTED = [
     "pf_kvbuf_bytes", "pf_create", "pf_destroy", "pf_kvbuf_init", "pf_patch_attn_step",
-    "pf_get_state", "pf_set_state", "pf_cfg_workspace_bytes", "pf_cfg_combine_relmae",
+    "pf_get_state", "pf_set_state", "pf_workspace_bytes", "pf_set_workspace",
+    "pf_cfg_workspace_bytes", "pf_cfg_combine_relmae",
     "pf_check_device_status", "pf_status_string", "pf_version",
 ]
 
@@ -72,6 +73,8 @@ def _lib():
             "pf_kvbuf_init": (i, [vp, i, vp, vp, vp]),
             "pf_patch_attn_step": (i, [vp, i, i, vp, vp, vp, vp, vp, vp, vp]),
             "pf_get_state": (i, [vp, i, ctypes.POINTER(i)]),
+            "pf_workspace_bytes": (sz, [cfgp]),
+            "pf_set_workspace": (i, [vp, vp, sz, vp]),
             "pf_set_state": (i, [vp, i, i]),
             "pf_cfg_workspace_bytes": (sz, [i, i64]),
             "pf_cfg_combine_relmae": (i, [vp, vp, i, i64, f, vp, vp, vp, vp, sz, vp]),
@@ -167,6 +170,18 @@ def pf_patch_attn_step(ctx, layer: int, patch: int, q_p, k_p, v_p, k_txt, v_txt,
            "pf_patch_attn_step")
 
 
+def pf_workspace_bytes(cfg: pf_config) -> int:
+    return int(_lib().pf_workspace_bytes(ctypes.byref(cfg)))
+
+
+def pf_set_workspace(ctx, ws: Optional[torch.Tensor], stream=None) -> None:
+    if ws is None:
+        _check(_lib().pf_set_workspace(ctx, None, 0, None), "pf_set_workspace")
+        return
+    ptr = _ptr(ws, torch.uint8, None, "workspace")
+    _check(_lib().pf_set_workspace(ctx, ptr, ws.numel(), _stream(stream)), "pf_set_workspace")
+
+
 def pf_get_state(ctx, layer: int) -> int:
     v = ctypes.c_int()
     _check(_lib().pf_get_state(ctx, layer, ctypes.byref(v)), "pf_get_state")
@@ -211,7 +226,7 @@ class PatchAttention:
     """
 
     def __init__(self, batch, heads, head_dim, n_img, n_patches, n_txt, n_layers,
-                 softmax_scale=0.0, schedule=PF_SCHED_PIPEFUSION, device="cuda"):
+                 softmax_scale=0.0, schedule=PF_SCHED_PIPEFUSION, device="cuda", split=True):
         self.cfg = make_config(batch, heads, head_dim, n_img, n_patches, n_txt, n_layers,
                                softmax_scale, schedule)
         nbytes = pf_kvbuf_bytes(self.cfg)
@@ -220,6 +235,11 @@ class PatchAttention:
         self.buffers: List[torch.Tensor] = [
             torch.empty(nbytes, dtype=torch.uint8, device=device) for _ in range(n_layers)]
         self.ctx = pf_create(self.cfg, [b.data_ptr() for b in self.buffers])
+        self.workspace = None
+        wsb = pf_workspace_bytes(self.cfg) if split else 0
+        if wsb > 0:
+            self.workspace = torch.empty(wsb, dtype=torch.uint8, device=device)
+            pf_set_workspace(self.ctx, self.workspace)
         self.plen = n_img // n_patches
         self.patch_shape = (batch, self.plen, heads, head_dim)
         self.full_shape = (batch, n_img, heads, head_dim)

@@ -24,6 +24,14 @@
 // maximum grows by more than 2^8, which is exact because the final O / l uses the same
 // reference maximum for numerator and denominator.
 //
+// Work decomposition: one CTA per (pair, part), where a pair is one (batch, head, group of
+// NQ query tiles) and its context tiles are split into n_split contiguous parts so that
+// the grid fills the SMs in near-whole waves.  A part that does not cover the whole
+// context writes its unnormalised O row with its reference maximum m and sum l to a
+// workspace slot; the last part of a query tile to finish (an atomic counter decides, no
+// CTA ever waits for another) merges all parts, O = sum_i 2^(m_i - M) O_i / sum_i 2^(m_i - M) l_i,
+// and writes the bf16 output.
+//
 // Every wait is bounded (2 s); on expiry the kernel records the role in a device word,
 // raises a CTA-wide abort flag, drains its in-flight copies and MMAs, frees TMEM and
 // returns.
@@ -50,6 +58,7 @@ constexpr int kWarpScatter = 10;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 256;        // O_t at column 256 + 128 t; S_t at column 128 t
 constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr int kMaxSplit = 16;          // most key-range parts per query tile
 
 enum : unsigned { kWdLoad = 1u, kWdMma = 2u, kWdSoftmax = 4u, kWdEpilogue = 8u };
 
@@ -111,6 +120,45 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// O row chunk of 16 fp32 columns (c0 .. c0+15) -> bf16, scaled by inv; columns >= D dropped.
+template <int D>
+__device__ __forceinline__ void store_row16(uint16_t* dst, int c0, const uint32_t (&o)[16], float inv,
+                                            bool in_range) {
+  uint4 w0, w1;
+  w0.x = pack_bf16(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);
+  w0.y = pack_bf16(__uint_as_float(o[2]) * inv, __uint_as_float(o[3]) * inv);
+  w0.z = pack_bf16(__uint_as_float(o[4]) * inv, __uint_as_float(o[5]) * inv);
+  w0.w = pack_bf16(__uint_as_float(o[6]) * inv, __uint_as_float(o[7]) * inv);
+  w1.x = pack_bf16(__uint_as_float(o[8]) * inv, __uint_as_float(o[9]) * inv);
+  w1.y = pack_bf16(__uint_as_float(o[10]) * inv, __uint_as_float(o[11]) * inv);
+  w1.z = pack_bf16(__uint_as_float(o[12]) * inv, __uint_as_float(o[13]) * inv);
+  w1.w = pack_bf16(__uint_as_float(o[14]) * inv, __uint_as_float(o[15]) * inv);
+  if (in_range) {
+    if (c0 + 8 <= D) *reinterpret_cast<uint4*>(dst + c0) = w0;
+    if (c0 + 16 <= D) *reinterpret_cast<uint4*>(dst + c0 + 8) = w1;
+  }
+}
+
+// Barrier among the `count` threads of one softmax warpgroup (ids 1 and 2; 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Barrier among `count` threads that also ANDs a predicate over them: every participant
+// gets the same answer, so a warpgroup agrees on whether to take a path with barriers.
+__device__ __forceinline__ bool named_bar_and(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ void raise_abort(volatile int* abort, unsigned code) {
   *abort = 1;
   atomicOr(&g_watchdog, code);
@@ -138,9 +186,13 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
-  const int q0 = blockIdx.x * NQ * kRows;
+  const int part = blockIdx.x / p.n_pairs;
+  const int pair = blockIdx.x - part * p.n_pairs;
+  const int grp = pair % p.n_groups;
+  const int h = (pair / p.n_groups) % p.heads;
+  const int b = pair / (p.n_groups * p.heads);
+  const int q0 = grp * NQ * kRows;
+  __shared__ int s_last[2];
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
@@ -180,7 +232,10 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
 
   Segments seg;
   seg.init(p);
-  const int n_tiles = seg.total();
+  const int n_all = seg.total();
+  const int j0 = static_cast<int>(static_cast<long long>(part) * n_all / p.n_split);
+  const int j1 = static_cast<int>(static_cast<long long>(part + 1) * n_all / p.n_split);
+  const int n_tiles = j1 - j0;  // this CTA's context tiles: j0 .. j1-1
 
   if (warp == kWarpLoad) {
     // ------------------------------------------------------------ TMA producer
@@ -195,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
       bool ok = true;
       for (int j = 0; j < n_tiles && ok; ++j) {
         int src, row0, nv;
-        seg.tile(j, src, row0, nv);
+        seg.tile(j0 + j, src, row0, nv);
         for (int kv = 0; kv < 2; ++kv) {
           const int i = 2 * j + kv;
           const int st = i % S;
@@ -292,34 +347,35 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
     }
   } else if (warp == kWarpScatter) {
     // ------------------------------------------------------------ buffer scatter
+    // Each CTA copies a contiguous 1/gridDim share of the flattened [B, P, H, d] fresh
+    // K and V into the buffer rows of the patch.
     if (p.k_dst != nullptr) {
-      constexpr int kVec = D / 8;  // 16-byte vectors per row of one head
-      const int r0 = q0;
-      const int r1 = min(q0 + NQ * kRows, p.plen);
-      const int total = (r1 - r0) * kVec;
-      const size_t src_row_stride = static_cast<size_t>(p.heads) * D;
-      const size_t dst_row0 = static_cast<size_t>(b) * p.n_img + static_cast<size_t>(p.patch) * p.plen;
+      const long long per_b = static_cast<long long>(p.plen) * p.heads * D / 8;  // 16-byte vectors
+      const long long total = per_b * p.batch;
+      const long long lo = total * blockIdx.x / gridDim.x;
+      const long long hi = total * (blockIdx.x + 1) / gridDim.x;
+      const long long img_b = static_cast<long long>(p.n_img) * p.heads * D / 8;
+      const long long patch_off = static_cast<long long>(p.patch) * per_b;
       const uint4* ksrc = reinterpret_cast<const uint4*>(p.k_p);
       const uint4* vsrc = reinterpret_cast<const uint4*>(p.v_p);
       uint4* kdst = reinterpret_cast<uint4*>(p.k_dst);
       uint4* vdst = reinterpret_cast<uint4*>(p.v_dst);
-      for (int base = lane; base < total; base += 32 * 4) {
+      for (long long base = lo + lane; base < hi; base += 32 * 4) {
         uint4 kx[4], vx[4];
-        size_t so[4], dof[4];
+        long long dof[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int i = base + u * 32;
-          if (i < total) {
-            const int r = r0 + i / kVec, v = i % kVec;
-            so[u] = ((static_cast<size_t>(b) * p.plen + r) * src_row_stride + static_cast<size_t>(h) * D) / 8 + v;
-            dof[u] = ((dst_row0 + r) * src_row_stride + static_cast<size_t>(h) * D) / 8 + v;
-            kx[u] = __ldg(ksrc + so[u]);
-            vx[u] = __ldg(vsrc + so[u]);
+          const long long i = base + u * 32;
+          if (i < hi) {
+            const long long bb = i / per_b;
+            dof[u] = bb * img_b + patch_off + (i - bb * per_b);
+            kx[u] = __ldg(ksrc + i);
+            vx[u] = __ldg(vsrc + i);
           }
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          if (base + u * 32 < total) {
+          if (base + u * 32 < hi) {
             kdst[dof[u]] = kx[u];
             vdst[dof[u]] = vx[u];
           }
@@ -349,15 +405,20 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
       tmem_ld32(tS + 96, s + 96);
       tmem_wait_ld();
       reg_fence<128>(s);
-      const int nv = seg.nvalid(j);
+      const int nv = seg.nvalid(j0 + j);
       if (nv < kRows) {
 #pragma unroll
         for (int k = 0; k < 128; ++k)
           if (k >= nv) s[k] = __float_as_uint(-INFINITY);
       }
-      float mx = __uint_as_float(s[0]);
+      // row maximum: 8 independent chains, then a tree
+      float mv[8];
 #pragma unroll
-      for (int k = 1; k < 128; ++k) mx = fmaxf(mx, __uint_as_float(s[k]));
+      for (int k = 0; k < 8; ++k) mv[k] = __uint_as_float(s[k]);
+#pragma unroll
+      for (int k = 8; k < 128; ++k) mv[k & 7] = fmaxf(mv[k & 7], __uint_as_float(s[k]));
+      const float mx = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
+                             fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
       const float mxs = mx * c;
       if (mxs > m + 8.f) {
         const float alpha = ex2(m - mxs);
@@ -378,50 +439,108 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
       }
       const float nm = -m;
       uint32_t pk[64];
+      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int k = 0; k < 64; ++k) {
         const float p0 = ex2(fmaf(__uint_as_float(s[2 * k]), c, nm));
         const float p1 = ex2(fmaf(__uint_as_float(s[2 * k + 1]), c, nm));
-        l += p0 + p1;
+        ls[k & 7] += p0 + p1;
         pk[k] = pack_bf16(p0, p1);
       }
+      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       tmem_st32(tS, pk);
       tmem_st32(tS + 32, pk + 32);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(p_full + t));
     }
-    if (!ok) {
-      if (lane == 0) raise_abort(abort, kWdSoftmax);
-    } else {
-      ok = mbar_wait(smem_u32(o_full + t), 0, abort, kWaitNs);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) {
-        if (lane == 0) raise_abort(abort, kWdEpilogue);
+    if (!ok && lane == 0) raise_abort(abort, kWdSoftmax);
+    {
+      bool ok_o = ok && mbar_wait(smem_u32(o_full + t), 0, abort, kWaitNs);
+      ok_o = __all_sync(0xffffffffu, ok_o);
+      // the whole warpgroup takes the same branch (the merge path has barriers)
+      ok_o = named_bar_and(1 + t, kRows, ok_o);
+      if (!ok_o) {
+        if (ok && lane == 0) raise_abort(abort, kWdEpilogue);
       } else {
         tc_fence_after();
-        const int row = q0 + t * kRows + wq * 32 + lane;
-        const float inv = 1.f / l;
+        const int rloc = wq * 32 + lane;
+        const int row = q0 + t * kRows + rloc;
         uint16_t* dst = p.o + ((static_cast<size_t>(b) * p.plen + row) * p.heads + h) * D;
         const bool in_range = row < p.plen;
+        if (p.n_split == 1) {
+          const float inv = 1.f / l;
 #pragma unroll
-        for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
-          uint32_t o[16];
-          tmem_ld16(tO + c0, o);
-          tmem_wait_ld();
-          reg_fence<16>(o);
-          uint4 w0, w1;
-          w0.x = pack_bf16(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);
-          w0.y = pack_bf16(__uint_as_float(o[2]) * inv, __uint_as_float(o[3]) * inv);
-          w0.z = pack_bf16(__uint_as_float(o[4]) * inv, __uint_as_float(o[5]) * inv);
-          w0.w = pack_bf16(__uint_as_float(o[6]) * inv, __uint_as_float(o[7]) * inv);
-          w1.x = pack_bf16(__uint_as_float(o[8]) * inv, __uint_as_float(o[9]) * inv);
-          w1.y = pack_bf16(__uint_as_float(o[10]) * inv, __uint_as_float(o[11]) * inv);
-          w1.z = pack_bf16(__uint_as_float(o[12]) * inv, __uint_as_float(o[13]) * inv);
-          w1.w = pack_bf16(__uint_as_float(o[14]) * inv, __uint_as_float(o[15]) * inv);
-          if (in_range) {
-            if (c0 + 8 <= D) *reinterpret_cast<uint4*>(dst + c0) = w0;
-            if (c0 + 16 <= D) *reinterpret_cast<uint4*>(dst + c0 + 8) = w1;
+          for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
+            uint32_t o[16];
+            tmem_ld16(tO + c0, o);
+            tmem_wait_ld();
+            reg_fence<16>(o);
+            store_row16<D>(dst, c0, o, inv, in_range);
+          }
+        } else {
+          // partial: O row (d columns), m, l into this part's slot, column-major
+          const size_t slot_elems = static_cast<size_t>(D + 2) * kRows;
+          float* slot0 = p.ws_part + (static_cast<size_t>(pair) * 2 + t) * p.n_split * slot_elems;
+          float* mine = slot0 + static_cast<size_t>(part) * slot_elems;
+#pragma unroll
+          for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
+            uint32_t o[16];
+            tmem_ld16(tO + c0, o);
+            tmem_wait_ld();
+            reg_fence<16>(o);
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+              if (c0 + k < D) mine[(c0 + k) * kRows + rloc] = __uint_as_float(o[k]);
+          }
+          mine[D * kRows + rloc] = m;
+          mine[(D + 1) * kRows + rloc] = l;
+          __threadfence();
+          named_bar_sync(1 + t, kRows);
+          if (rloc == 0) {
+            const unsigned old = atomicAdd(p.ws_cnt + pair * 2 + t, 1u);
+            const int last = old == static_cast<unsigned>(p.n_split - 1);
+            if (last) {
+              __threadfence();
+              p.ws_cnt[pair * 2 + t] = 0u;  // ready for the next launch
+            }
+            s_last[t] = last;
+          }
+          named_bar_sync(1 + t, kRows);
+          if (s_last[t]) {
+            // merge every part of this query tile
+            float wgt[kMaxSplit];
+            float mref = -INFINITY;
+            for (int i = 0; i < p.n_split; ++i)
+              mref = fmaxf(mref, __ldcg(slot0 + i * slot_elems + D * kRows + rloc));
+            float lsum = 0.f;
+            for (int i = 0; i < kMaxSplit; ++i) {
+              if (i < p.n_split) {
+                const float* si = slot0 + i * slot_elems;
+                wgt[i] = ex2(__ldcg(si + D * kRows + rloc) - mref);
+                lsum += wgt[i] * __ldcg(si + (D + 1) * kRows + rloc);
+              } else {
+                wgt[i] = 0.f;
+              }
+            }
+            const float inv = 1.f / lsum;
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 8) {
+              float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+              for (int i = 0; i < p.n_split; ++i) {
+                const float* si = slot0 + i * slot_elems + c0 * kRows + rloc;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) acc[k] += wgt[i] * __ldcg(si + k * kRows);
+              }
+              if (in_range) {
+                uint4 w0;
+                w0.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+                w0.y = pack_bf16(acc[2] * inv, acc[3] * inv);
+                w0.z = pack_bf16(acc[4] * inv, acc[5] * inv);
+                w0.w = pack_bf16(acc[6] * inv, acc[7] * inv);
+                *reinterpret_cast<uint4*>(dst + c0) = w0;
+              }
+            }
           }
         }
       }
@@ -446,12 +565,60 @@ cudaError_t launch_one(const AttnParams& p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  dim3 grid((p.plen + NQ * kRows - 1) / (NQ * kRows), p.heads, p.batch);
+  const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.n_split);
   patch_attn_kernel<D, NQ><<<grid, kThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
+__global__ void zero_u32_kernel(unsigned* p, size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    p[i] = 0u;
+}
+
 }  // namespace
+
+int attn_tiles_per_cta(int plen) { return plen > kRows ? 2 : 1; }
+
+int attn_context_tiles(int plen, int n_img, int n_txt, int patch) {
+  auto tiles = [](long long n) { return static_cast<int>((n + kRows - 1) / kRows); };
+  return tiles(plen) + tiles(static_cast<long long>(patch) * plen) +
+         tiles(n_img - static_cast<long long>(patch + 1) * plen) + tiles(n_txt);
+}
+
+int attn_choose_split(int n_pairs, int n_tiles, int n_sms, int max_split) {
+  // cost model in units of context tiles: whole waves of CTAs times the tiles per CTA plus
+  // a fixed per-CTA overhead (launch, TMEM allocation, Q load, pipeline fill, merge)
+  constexpr long long kOverheadTiles = 6;
+  int best = 1;
+  long long best_cost = -1;
+  const int kmax = max_split < kMaxSplit ? max_split : kMaxSplit;
+  for (int k = 1; k <= kmax && k <= n_tiles; ++k) {
+    const long long ctas = static_cast<long long>(n_pairs) * k;
+    const long long waves = (ctas + n_sms - 1) / n_sms;
+    const long long cost = waves * ((n_tiles + k - 1) / k + kOverheadTiles);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = k;
+    }
+  }
+  return best;
+}
+
+size_t attn_workspace_bytes(int n_pairs, int head_dim, int n_split) {
+  if (n_split <= 1) return 0;
+  const size_t part_bytes = static_cast<size_t>(n_pairs) * 2 * n_split * (head_dim + 2) * kRows * 4;
+  const size_t cnt_bytes = static_cast<size_t>(n_pairs) * 2 * 4;
+  return ((part_bytes + 255) / 256) * 256 + cnt_bytes;
+}
+
+cudaError_t launch_zero_u32(unsigned* p, size_t n, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  size_t blocks = (n + 255) / 256;
+  if (blocks > 1024) blocks = 1024;
+  zero_u32_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p, n);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_patch_attn(const AttnParams& p, cudaStream_t stream) {
   const bool two = p.plen > kRows;

@@ -26,6 +26,9 @@ struct pf_ctx {
   std::vector<int> read_half;    // DistriFusion: which half of the buffer holds the stale step
   std::vector<std::vector<uint8_t>> seen;  // DistriFusion: patches done in the current step
   std::vector<int> seen_count;
+  uint8_t* ws = nullptr;         // optional attention workspace (caller-owned)
+  size_t ws_bytes = 0;
+  int n_sms = 0;                 // queried on first use
 };
 
 namespace {
@@ -93,6 +96,32 @@ bool make_map(CUtensorMap* m, const void* base, int batch, int rows, int heads, 
 }
 
 pf_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PF_OK : PF_ERR_CUDA; }
+
+int pairs_of(const pf_config& c) {
+  const int plen = c.n_img / c.n_patches;
+  const int nq = pf::attn_tiles_per_cta(plen);
+  const int groups = (plen + nq * 128 - 1) / (nq * 128);
+  return c.batch * c.heads * groups;
+}
+
+constexpr int kAssumedSms = 148;
+
+// Counters first (fixed place), then the partial slots.
+size_t counter_bytes(int pairs) { return ((static_cast<size_t>(pairs) * 2 * 4 + 255) / 256) * 256; }
+
+size_t workspace_for(const pf_config& c, int n_sms) {
+  const int plen = c.n_img / c.n_patches;
+  const int pairs = pairs_of(c);
+  size_t best = 0;
+  for (int p = 0; p < c.n_patches; ++p) {
+    const int tiles = pf::attn_context_tiles(plen, c.n_img, c.n_txt, p);
+    const int k = pf::attn_choose_split(pairs, tiles, n_sms, 1 << 30);
+    const size_t b = k > 1 ? counter_bytes(pairs) + pf::attn_workspace_bytes(pairs, c.head_dim, k) : 0;
+    if (b > best) best = b;
+    if (plen % 128 == 0) break;  // every patch has the same tile count
+  }
+  return best;
+}
 
 bool layer_ok(const pf_ctx* ctx, int layer) { return layer >= 0 && layer < ctx->cfg.n_layers; }
 
@@ -209,6 +238,29 @@ pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
   p.patch = patch;
   p.head_dim = d;
   p.scale_log2 = ctx->scale * 1.4426950408889634f;
+  const int nq = pf::attn_tiles_per_cta(plen);
+  p.n_groups = (plen + nq * 128 - 1) / (nq * 128);
+  p.n_pairs = c.batch * c.heads * p.n_groups;
+  p.n_split = 1;
+  if (ctx->ws != nullptr) {
+    if (ctx->n_sms == 0) {
+      int dev = 0, n = 0;
+      if (cudaGetDevice(&dev) == cudaSuccess &&
+          cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+        ctx->n_sms = n;
+      else
+        ctx->n_sms = kAssumedSms;
+    }
+    const int tiles = pf::attn_context_tiles(plen, c.n_img, c.n_txt, patch);
+    const size_t cb = counter_bytes(p.n_pairs);
+    int cap = 1;  // most parts the workspace can hold
+    while (cap < 16 && cb + pf::attn_workspace_bytes(p.n_pairs, d, cap + 1) <= ctx->ws_bytes) ++cap;
+    p.n_split = pf::attn_choose_split(p.n_pairs, tiles, ctx->n_sms, cap);
+    if (p.n_split > 1) {
+      p.ws_cnt = reinterpret_cast<unsigned*>(ctx->ws);
+      p.ws_part = reinterpret_cast<float*>(ctx->ws + cb);
+    }
+  }
 
   cudaError_t e = pf::launch_patch_attn(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return PF_ERR_CUDA;
@@ -242,6 +294,28 @@ pf_status pf_set_state(pf_ctx* ctx, int layer, int next_patch) {
   if (ctx->cfg.schedule != PF_SCHED_PIPEFUSION && next_patch != 0) return PF_ERR_UNSUPPORTED;
   ctx->next_patch[layer] = next_patch;
   ctx->initialised[layer] = 1;
+  return PF_OK;
+}
+
+size_t pf_workspace_bytes(const pf_config* cfg) {
+  if (check_config(cfg) != PF_OK) return 0;
+  return workspace_for(*cfg, kAssumedSms);
+}
+
+pf_status pf_set_workspace(pf_ctx* ctx, void* ws, size_t ws_bytes, void* stream) {
+  if (!ctx) return PF_ERR_INVALID_ARG;
+  if (ws == nullptr) {
+    ctx->ws = nullptr;
+    ctx->ws_bytes = 0;
+    return PF_OK;
+  }
+  if (!aligned16(ws)) return PF_ERR_ALIGN;
+  const size_t cb = counter_bytes(pairs_of(ctx->cfg));
+  if (ws_bytes < cb) return PF_ERR_INVALID_ARG;
+  cudaError_t e = pf::launch_zero_u32(static_cast<unsigned*>(ws), cb / 4, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return PF_ERR_CUDA;
+  ctx->ws = static_cast<uint8_t*>(ws);
+  ctx->ws_bytes = ws_bytes;
   return PF_OK;
 }
 

@@ -27,7 +27,26 @@ struct AttnParams {
   uint16_t* o;          // O_p [B, P, H, d]
   int batch, heads, plen, n_img, n_txt, patch, head_dim;
   float scale_log2;     // softmax scale * log2(e)
+  // Work decomposition: a "pair" is one (batch, head, group of NQ query tiles); its key
+  // range is split into n_split contiguous parts, one CTA per (pair, part).
+  int n_groups;         // query-tile groups per (batch, head)
+  int n_pairs;          // batch * heads * n_groups
+  int n_split;          // parts per pair (1 => no partials)
+  float* ws_part;       // partial (O, m, l) slots, [pair][tile][part][d + 2][128] fp32
+  unsigned* ws_cnt;     // finished-part counters, [pair][tile]; zero between launches
 };
+
+// Query tiles per CTA chosen for a patch length (1 or 2).
+int attn_tiles_per_cta(int plen);
+// Number of 128-row context tiles of one micro-step.
+int attn_context_tiles(int plen, int n_img, int n_txt, int patch);
+// Key-range parts per (batch, head, query-tile group) for a call, given the number of SMs
+// and the number of parts the workspace can hold.
+int attn_choose_split(int n_pairs, int n_tiles, int n_sms, int max_split);
+// Workspace bytes for n_pairs pairs split into n_split parts.
+size_t attn_workspace_bytes(int n_pairs, int head_dim, int n_split);
+// Zero the counters of a workspace.
+cudaError_t launch_zero_u32(unsigned* p, size_t n, cudaStream_t stream);
 
 // Launch the fused scatter + attention kernel.  Returns the launch error.
 cudaError_t launch_patch_attn(const AttnParams& p, cudaStream_t stream);

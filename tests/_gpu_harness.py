@@ -78,7 +78,8 @@ def vmax_used(cur_cpu, prev_cpu, p, n_patches, b=0, heads=None):
 
 def run_workload(wl: synth.AttnWorkload, steps: Optional[int] = None, full_check=lambda s, l, p: True,
                  sample_check=lambda s, l, p: False, n_sample_rows: int = 8, seed: Optional[int] = None,
-                 schedule=pa.PF_SCHED_PIPEFUSION, a=None, b=None, oracle_buffer=lambda s, l, p: False):
+                 schedule=pa.PF_SCHED_PIPEFUSION, a=None, b=None, oracle_buffer=lambda s, l, p: False,
+                 split=True):
     """Run `steps` diffusion steps of `wl` through the library and check against the oracle.
 
     full_check(s, l, p)   -> compare every output row of that call with the oracle
@@ -89,7 +90,7 @@ def run_workload(wl: synth.AttnWorkload, steps: Optional[int] = None, full_check
     S = wl.n_steps if steps is None else steps
     gen = synth.AttnInputs(wl, seed=seed, device=dev, a=a, b=b)
     pat = pa.PatchAttention(wl.batch, wl.heads, wl.head_dim, wl.n_img, wl.n_patches, wl.n_txt,
-                            wl.n_layers, schedule=schedule)
+                            wl.n_layers, schedule=schedule, split=split)
     rng = np.random.default_rng(1234)
     chk = Checker()
     P = wl.patch_len

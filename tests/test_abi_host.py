@@ -164,3 +164,20 @@ def test_cfg_argument_checks():
     assert call(u=FAKE + 4) == pa.PF_ERR_ALIGN
     assert call(ob=FAKE + 2) == pa.PF_ERR_ALIGN
     assert call(wsb=ws - 1) == pa.PF_ERR_INVALID_ARG
+
+
+def test_workspace_sizes_and_checks():
+    # SD3-like call: 192 query-tile pairs; the split needs counters + partial slots
+    c = _cfg(heads=24, n_img=16384, n_patches=8, n_txt=154, head_dim=64, n_layers=1)
+    ws = pa.pf_workspace_bytes(c)
+    assert ws > 192 * 2 * 4
+    assert pa.pf_workspace_bytes(_cfg(head_dim=96)) == 0
+    ctx = pa.pf_create(c, [FAKE])
+    try:
+        L = pa._lib()
+        assert L.pf_set_workspace(ctx, FAKE + 8, ws, None) == pa.PF_ERR_ALIGN
+        assert L.pf_set_workspace(ctx, FAKE, 16, None) == pa.PF_ERR_INVALID_ARG
+        assert L.pf_set_workspace(ctx, None, 0, None) == pa.PF_OK
+        assert L.pf_set_workspace(None, FAKE, ws, None) == pa.PF_ERR_INVALID_ARG
+    finally:
+        pa.pf_destroy(ctx)

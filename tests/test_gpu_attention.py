@@ -59,12 +59,15 @@ def test_flux_full_size_sampled():
     assert chk.n > 0
 
 
+@pytest.mark.parametrize("split", [True, False])
 @pytest.mark.parametrize("d", [64, 72, 128])
-def test_ragged_shapes(d):
-    # patches that are not multiples of the 128-row tile, a ragged text tail, batch 2
+def test_ragged_shapes(d, split):
+    # patches that are not multiples of the 128-row tile, a ragged text tail, batch 2;
+    # with and without the key-range split across CTAs
     wl = synth.AttnWorkload("ragged", batch=2, heads=3, head_dim=d, grid_h=20, grid_w=30,
                             n_patches=3, n_txt=77, n_layers=2, n_steps=3, ar_a=0.95, ar_b=0.3)
-    chk = run_workload(wl, full_check=lambda s, l, p: True, oracle_buffer=lambda s, l, p: True)
+    chk = run_workload(wl, full_check=lambda s, l, p: True, oracle_buffer=lambda s, l, p: True,
+                       split=split)
     assert chk.n == 3 * 2 * 3 * 2
 
 
