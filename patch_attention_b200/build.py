@@ -35,16 +35,21 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) -> str:
-    os.makedirs(OBJDIR, exist_ok=True)
+def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True,
+          trace: bool = False) -> str:
+    """trace=True builds libpatchattn_trace.so with per-tile timestamps of CTA 0 (profiling)."""
+    objdir = OBJDIR + ("_trace" if trace else "")
+    lib = LIB.replace(".so", "_trace.so") if trace else LIB
+    extra = ["-DPF_TRACE"] if trace else []
+    os.makedirs(objdir, exist_ok=True)
     hdrs = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(INCLUDE, "patchattn.h")]
     objs = []
     for src in SOURCES:
         path = os.path.join(CSRC, src)
-        obj = os.path.join(OBJDIR, src + ".o")
+        obj = os.path.join(objdir, src + ".o")
         objs.append(obj)
         if force or _stale(obj, [path] + hdrs):
-            cmd = [NVCC] + ARCH + COMMON + ["-c", path, "-o", obj]
+            cmd = [NVCC] + ARCH + COMMON + extra + ["-c", path, "-o", obj]
             if ptxas_verbose and src.endswith(".cu"):
                 cmd += ["-Xptxas", "-v"]
             if src.endswith(".cpp"):
@@ -54,18 +59,19 @@ def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) 
                 sys.stderr.write(r.stdout + r.stderr)
             if r.returncode != 0:
                 raise RuntimeError(f"nvcc failed on {src}")
-    if force or _stale(LIB, objs):
-        cmd = [NVCC] + ARCH + ["-shared", "-cudart", "static", "-o", LIB] + objs
+    if force or _stale(lib, objs):
+        cmd = [NVCC] + ARCH + ["-shared", "-cudart", "static", "-o", lib] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)
             raise RuntimeError("link failed")
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--ptxas-verbose", action="store_true")
+    ap.add_argument("--trace", action="store_true")
     a = ap.parse_args()
-    print(build(force=a.force, ptxas_verbose=a.ptxas_verbose, quiet=not a.ptxas_verbose))
+    print(build(force=a.force, ptxas_verbose=a.ptxas_verbose, quiet=not a.ptxas_verbose, trace=a.trace))

@@ -45,13 +45,38 @@ namespace pf {
 
 __device__ unsigned int g_watchdog = 0;
 
+#ifdef PF_TRACE
+// Profiling build only: SM-cycle timestamps of CTA 0, [event][query tile][context tile].
+// Events: 0 softmax sees S, 1 softmax has published P, 2 MMA issuer sees P,
+// 3 MMA issuer has committed S, 4 MMA issuer sees the K tile, 5 softmax has S in
+// registers, 6 softmax has the row maximum, 7 softmax has P packed, 8 P stored to TMEM.
+constexpr int kTraceTiles = 512;
+// 9 MMA issuer sees the V tile of j-1, 10 producer issued the K (t=0) / V (t=1) tile j.
+__device__ unsigned long long g_trace[11 * 2 * kTraceTiles];
+#define PF_TRACE_AT(ev, t, j)                                                              \
+  do {                                                                                     \
+    if (blockIdx.x == 0 && (j) < kTraceTiles) g_trace[((ev) * 2 + (t)) * kTraceTiles + (j)] = clock64(); \
+  } while (0)
+#else
+#define PF_TRACE_AT(ev, t, j) \
+  do {                        \
+  } while (0)
+#endif
+
 namespace {
 
 using namespace ptx;
 
 constexpr int kRows = 128;             // query rows per Q tile == key rows per K/V tile
 constexpr int kChunkBytes = 128 * 128; // 128 rows x 64 bf16 columns (one 128-byte swizzle span)
-constexpr int kThreads = 352;          // 11 warps
+constexpr int kThreads = 384;          // 3 warpgroups: softmax 0, softmax 1, MMA/TMA/scatter
+// Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512), the third
+// warpgroup drops to 88 and the two softmax warpgroups rise to 208:
+// 128 x 88 + 256 x 208 = 64512, exactly the registers the CTA was launched with.  (88 keeps
+// the MMA issuer free of spills; 56/224 measured slower.)
+constexpr uint32_t kRegsSoftmax = 208;
+constexpr uint32_t kRegsOther = 88;
+static_assert(128 * kRegsOther + 256 * kRegsSoftmax <= kThreads * 168, "register split");
 constexpr int kWarpMma = 8;
 constexpr int kWarpLoad = 9;
 constexpr int kWarpScatter = 10;
@@ -72,7 +97,7 @@ struct Dims {
 
 template <int D, int NQ>
 constexpr int smem_bytes() {
-  return 1024 + (NQ + Dims<D>::kStages) * Dims<D>::kTileBytes + 256;
+  return 1024 + (NQ + Dims<D>::kStages) * Dims<D>::kTileBytes + 512;
 }
 
 // Which tensor and rows the j-th 128-row context tile comes from.
@@ -159,6 +184,88 @@ __device__ __forceinline__ bool named_bar_and(int id, int count, bool pred) {
   return r != 0;
 }
 
+// 2^x on the FMA pipe: x = n + f with n = round(x) (1.5 * 2^23 shifter), 2^f from a
+// degree-3 polynomial fitted on [-1/2, 1/2] for least maximum relative error (7.5e-5,
+// Lawson's iteratively reweighted least squares), and n added to the exponent field.
+// x is clamped to >= -125 so the result stays normal; callers never pass masked (-inf)
+// logits here.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 sh = make_float2(12582912.f, 12582912.f);
+  const float2 t = __fadd2_rn(x, sh);                                     // 1.5 * 2^23 + round(x)
+  const float2 r = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));  // round(x), exact
+  const float2 f = __ffma2_rn(r, make_float2(-1.f, -1.f), x);             // x - round(x), exact
+  float2 p = __ffma2_rn(make_float2(0.05517132f, 0.05517132f), f, make_float2(0.24261054f, 0.24261054f));
+  p = __ffma2_rn(p, f, make_float2(0.69326097f, 0.69326097f));
+  p = __ffma2_rn(p, f, make_float2(0.99992812f, 0.99992812f));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// Maximum of 128 values: 8 independent chains, then a tree.
+__device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) {
+  float mv[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mv[k] = __uint_as_float(s[k]);
+#pragma unroll
+  for (int k = 8; k < 128; ++k) mv[k & 7] = fmaxf(mv[k & 7], __uint_as_float(s[k]));
+  return fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
+               fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
+}
+
+// p_k = 2^(s_k c - m) with the special-function unit, packed to bf16 pairs; returns the
+// fp32 sum.  Masked keys (-inf) give exactly 0.
+__device__ __forceinline__ void exact_exps(const uint32_t (&s)[128], float c, float m,
+                                           uint32_t (&pk)[64], float& lsum) {
+  const float2 cc = make_float2(c, c), nm = make_float2(-m, -m);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int k = 0; k < 64; ++k) {
+    const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), cc, nm);
+    const float2 p = make_float2(ex2(x.x), ex2(x.y));
+    acc[k & 3] = __fadd2_rn(acc[k & 3], p);
+    pk[k] = pack_bf16(p.x, p.y);
+  }
+  const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  lsum = a.x + a.y;
+}
+
+// Same as exact_exps against the current reference m, with POLY of every 8 pairs of
+// columns exponentiated on the FMA pipe; returns max_k (s_k c - m) so the caller can
+// check that no p_k exceeded 2^8.
+template <int POLY>
+__device__ __forceinline__ float speculative_exps(const uint32_t (&s)[128], float c, float m,
+                                                  uint32_t (&pk)[64], float& lsum) {
+  const float2 cc = make_float2(c, c), nm = make_float2(-m, -m);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
+  float xm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int k = 0; k < 64; ++k) {
+    const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), cc, nm);
+    xm[k & 3] = fmaxf(xm[k & 3], fmaxf(x.x, x.y));
+    float2 p;
+    if ((k & 7) < POLY) {
+      p = exp2_poly2(x);
+    } else {
+      p = make_float2(ex2(x.x), ex2(x.y));
+    }
+    acc[k & 3] = __fadd2_rn(acc[k & 3], p);
+    pk[k] = pack_bf16(p.x, p.y);
+  }
+  const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  lsum = a.x + a.y;
+  return fmaxf(fmaxf(xm[0], xm[1]), fmaxf(xm[2], xm[3]));
+}
+
+// Of every 8 pairs of columns, the pairs whose exponentials run on the FMA pipe instead of
+// the special-function unit (3/8: balances the unit's 16 results/clk/SM against the extra
+// issue slots of the polynomial, about 5 instructions per element).
+template <int D>
+constexpr int kPolyPairs = 3;
+
 __device__ __forceinline__ void raise_abort(volatile int* abort, unsigned code) {
   *abort = 1;
   atomicOr(&g_watchdog, code);
@@ -202,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(smem_u32(s_full + t), 1);
-      mbar_init(smem_u32(p_full + t), kRows);
+      mbar_init(smem_u32(p_full + t), 4);  // one arrival per softmax warp
       mbar_init(smem_u32(o_full + t), 1);
     }
     mbar_init(smem_u32(mma_done), 1);
@@ -237,6 +344,10 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
   const int j1 = static_cast<int>(static_cast<long long>(part + 1) * n_all / p.n_split);
   const int n_tiles = j1 - j0;  // this CTA's context tiles: j0 .. j1-1
 
+  if (warp >= 8) {
+  // Every warp of a warpgroup executes the same setmaxnreg, inside the branch whose code
+  // runs under that register budget.
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
   if (warp == kWarpLoad) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -267,6 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
             tma_load_4d(smem_u32(sKV + st * Dm::kTileBytes + c * kChunkBytes), m, c * 64, h, row0,
                         b, fb);
           issued = i + 1;
+          PF_TRACE_AT(10, kv, j);
         }
       }
       if (!ok) raise_abort(abort, kWdLoad);
@@ -283,23 +395,28 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
       const uint32_t q_base = smem_u32(sQ);
       const uint32_t kv_base = smem_u32(sKV);
 
+      // Base descriptors are built once; an operand at byte offset `off` from a base only
+      // changes the 14-bit start-address field, by off >> 4 (no carry: smem < 256 KB).
+      const uint64_t dq0 = smem_desc_sw128(q_base, 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(kv_base, 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(kv_base, kChunkBytes, 1024);
       auto issue_qk = [&](int t, int st) {
-        const uint32_t a0 = q_base + t * Dm::kTileBytes;
-        const uint32_t b0 = kv_base + st * Dm::kTileBytes;
+        const uint64_t a0 = dq0 + static_cast<uint64_t>((t * Dm::kTileBytes) >> 4);
+        const uint64_t b0 = dk0 + static_cast<uint64_t>((st * Dm::kTileBytes) >> 4);
+        const uint32_t d = tmem + t * 128;
 #pragma unroll
         for (int kk = 0; kk < Dm::kMmaN / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-          mma_ss(tmem + t * 128, smem_desc_sw128(a0 + off, 16, 1024),
-                 smem_desc_sw128(b0 + off, 16, 1024), idesc_qk, kk > 0);
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+          mma_ss(d, a0 + off, b0 + off, idesc_qk, kk > 0);
         }
       };
       auto issue_pv = [&](int t, int st, bool acc) {
-        const uint32_t v0 = kv_base + st * Dm::kTileBytes;
+        const uint64_t v0 = dv0 + static_cast<uint64_t>((st * Dm::kTileBytes) >> 4);
+        const uint32_t d = tmem + kColO + t * 128;
+        const uint32_t a = tmem + t * 128;
 #pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk) {
-          mma_ts(tmem + kColO + t * 128, tmem + t * 128 + kk * 8,
-                 smem_desc_sw128(v0 + kk * 2048, kChunkBytes, 1024), idesc_pv, acc || kk > 0);
-        }
+        for (int kk = 0; kk < kRows / 16; ++kk)
+          mma_ts(d, a + kk * 8, v0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv, acc || kk > 0);
       };
 
       bool ok = mbar_wait(smem_u32(q_full), 0, abort, kWaitNs);
@@ -308,21 +425,25 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
         const int iK = 2 * j, sK = iK % S;
         if (!(ok = mbar_wait(smem_u32(kv_full + sK), (iK / S) & 1, abort, kWaitNs))) break;
         tc_fence_after();
+        PF_TRACE_AT(4, 0, j);
         int sV = 0;
         if (j > 0) {
           const int iV = 2 * j - 1;
           sV = iV % S;
           if (!(ok = mbar_wait(smem_u32(kv_full + sV), (iV / S) & 1, abort, kWaitNs))) break;
+          PF_TRACE_AT(9, 0, j - 1);
           tc_fence_after();
         }
         for (int t = 0; t < NQ; ++t) {
           if (j > 0) {
             if (!(ok = mbar_wait(smem_u32(p_full + t), (j - 1) & 1, abort, kWaitNs))) break;
             tc_fence_after();
+            PF_TRACE_AT(2, t, j - 1);
             issue_pv(t, sV, j - 1 > 0);
           }
           issue_qk(t, sK);
           mma_commit(smem_u32(s_full + t));
+          PF_TRACE_AT(3, t, j);
         }
         if (!ok) break;
         mma_commit(smem_u32(kv_empty + sK));
@@ -360,29 +481,32 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
       const uint4* vsrc = reinterpret_cast<const uint4*>(p.v_p);
       uint4* kdst = reinterpret_cast<uint4*>(p.k_dst);
       uint4* vdst = reinterpret_cast<uint4*>(p.v_dst);
-      for (long long base = lo + lane; base < hi; base += 32 * 4) {
-        uint4 kx[4], vx[4];
-        long long dof[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const long long i = base + u * 32;
-          if (i < hi) {
-            const long long bb = i / per_b;
-            dof[u] = bb * img_b + patch_off + (i - bb * per_b);
-            kx[u] = __ldg(ksrc + i);
-            vx[u] = __ldg(vsrc + i);
+      // walk the share one batch element at a time: within one, the destination is the
+      // source index shifted by a constant
+      for (long long bb = lo / per_b; bb * per_b < hi; ++bb) {
+        const long long b_lo = bb * per_b > lo ? bb * per_b : lo;
+        const long long b_hi = (bb + 1) * per_b < hi ? (bb + 1) * per_b : hi;
+        const long long shift = bb * (img_b - per_b) + patch_off;
+        for (long long base = b_lo + lane; base < b_hi; base += 32 * 2) {
+          const long long i1 = base + 32;
+          const uint4 k0 = __ldg(ksrc + base), v0 = __ldg(vsrc + base);
+          uint4 k1, v1;
+          if (i1 < b_hi) {
+            k1 = __ldg(ksrc + i1);
+            v1 = __ldg(vsrc + i1);
           }
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (base + u * 32 < hi) {
-            kdst[dof[u]] = kx[u];
-            vdst[dof[u]] = vx[u];
+          kdst[base + shift] = k0;
+          vdst[base + shift] = v0;
+          if (i1 < b_hi) {
+            kdst[i1 + shift] = k1;
+            vdst[i1 + shift] = v1;
           }
         }
       }
     }
+  }
   } else if (warp < 4 * NQ) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ------------------------------------------------------------ softmax + epilogue
     const int t = warp >> 2;
     const int wq = warp & 3;
@@ -398,6 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
+      if (wq == 0 && lane == 0) PF_TRACE_AT(0, t, j);
       uint32_t s[128];
       tmem_ld32(tS + 0, s);
       tmem_ld32(tS + 32, s + 32);
@@ -405,54 +530,64 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
       tmem_ld32(tS + 96, s + 96);
       tmem_wait_ld();
       reg_fence<128>(s);
+      if (wq == 0 && lane == 0) PF_TRACE_AT(5, t, j);
       const int nv = seg.nvalid(j0 + j);
-      if (nv < kRows) {
-#pragma unroll
-        for (int k = 0; k < 128; ++k)
-          if (k >= nv) s[k] = __float_as_uint(-INFINITY);
-      }
-      // row maximum: 8 independent chains, then a tree
-      float mv[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mv[k] = __uint_as_float(s[k]);
-#pragma unroll
-      for (int k = 8; k < 128; ++k) mv[k & 7] = fmaxf(mv[k & 7], __uint_as_float(s[k]));
-      const float mx = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
-                             fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
-      const float mxs = mx * c;
-      if (mxs > m + 8.f) {
-        const float alpha = ex2(m - mxs);
-        l *= alpha;
-        if (j > 0) {
-#pragma unroll
-          for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
-            uint32_t o[16];
-            tmem_ld16(tO + c0, o);
-            tmem_wait_ld();
-            reg_fence<16>(o);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st16(tO + c0, o);
-          }
-        }
-        m = mxs;
-      }
-      const float nm = -m;
       uint32_t pk[64];
-      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int k = 0; k < 64; ++k) {
-        const float p0 = ex2(fmaf(__uint_as_float(s[2 * k]), c, nm));
-        const float p1 = ex2(fmaf(__uint_as_float(s[2 * k + 1]), c, nm));
-        ls[k & 7] += p0 + p1;
-        pk[k] = pack_bf16(p0, p1);
+      float lsum;
+      // Fast path: exponentiate against the current reference maximum m straight away and
+      // check afterwards that no value exceeded 2^8; the row maximum is then off the
+      // critical path.  The first tile (no reference yet), ragged tiles (masked keys) and
+      // the rare tile whose maximum grew by more than 2^8 take the exact path instead.
+      bool exact = (j == 0) || (nv < kRows);
+      if (!exact) {
+        float xm = speculative_exps<kPolyPairs<D>>(s, c, m, pk, lsum);
+        if (xm > 8.f) {
+          // S is still in TMEM (P has not been written yet): reload it for the exact path
+          exact = true;
+          tmem_ld32(tS + 0, s);
+          tmem_ld32(tS + 32, s + 32);
+          tmem_ld32(tS + 64, s + 64);
+          tmem_ld32(tS + 96, s + 96);
+          tmem_wait_ld();
+          reg_fence<128>(s);
+        }
       }
-      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+      if (exact) {
+        if (nv < kRows) {
+#pragma unroll
+          for (int k = 0; k < 128; ++k)
+            if (k >= nv) s[k] = __float_as_uint(-INFINITY);
+        }
+        const float mxs = row_max128(s) * c;
+        if (mxs > m + 8.f) {
+          const float alpha = ex2(m - mxs);
+          l *= alpha;
+          if (j > 0) {
+#pragma unroll
+            for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
+              uint32_t o[16];
+              tmem_ld16(tO + c0, o);
+              tmem_wait_ld();
+              reg_fence<16>(o);
+#pragma unroll
+              for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+              tmem_st16(tO + c0, o);
+            }
+          }
+          m = mxs;
+        }
+        exact_exps(s, c, m, pk, lsum);
+      }
+      l += lsum;
+      if (wq == 0 && lane == 0) PF_TRACE_AT(7, t, j);
       tmem_st32(tS, pk);
       tmem_st32(tS + 32, pk + 32);
       tmem_wait_st();
+      if (wq == 0 && lane == 0) PF_TRACE_AT(8, t, j);
       tc_fence_before();
-      mbar_arrive(smem_u32(p_full + t));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(p_full + t));
+      if (wq == 0 && lane == 0) PF_TRACE_AT(1, t, j);
     }
     if (!ok && lane == 0) raise_abort(abort, kWdSoftmax);
     {
@@ -545,6 +680,9 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
         }
       }
     }
+  } else {
+    // second softmax warpgroup when the CTA has a single query tile: idle
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
   }
 
   tc_fence_before();
@@ -629,6 +767,13 @@ cudaError_t launch_patch_attn(const AttnParams& p, cudaStream_t stream) {
     default: return cudaErrorInvalidValue;
   }
 }
+
+#ifdef PF_TRACE
+extern "C" int pf_trace_read(unsigned long long* dst, size_t n) {
+  if (n > sizeof(g_trace) / sizeof(g_trace[0])) n = sizeof(g_trace) / sizeof(g_trace[0]);
+  return static_cast<int>(cudaMemcpyFromSymbol(dst, g_trace, n * sizeof(unsigned long long)));
+}
+#endif
 
 cudaError_t read_and_clear_watchdog(unsigned* value) {
   unsigned v = 0;
