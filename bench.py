@@ -400,7 +400,7 @@ def run_gpu(args, world, rank, local):
 
 def measure_cfg_largest(pa, dev, hbm, reps: int = 20):
     """The guidance kernel alone at the largest sweep size (batch 4 x 16x512x512, fp32 and bf16
-    outputs: 8 B read + 6 B written per element), L2 flushed (a 256 MB write) before each
+    outputs: 8 B read + 6 B written per element), L2 flushed (a 512 MB read) before each
     timed call; median of `reps` calls timed with CUDA events."""
     wl = synth.CfgWorkload("cfg", 4, 16, 512, 512)
     c, u = synth.CfgInputs(wl, device=dev).step_tensors(25)
@@ -409,11 +409,12 @@ def measure_cfg_largest(pa, dev, hbm, reps: int = 20):
     out_b = torch.empty(c.shape, dtype=torch.bfloat16, device=dev)
     rel = torch.empty(wl.batch, dtype=torch.float32, device=dev)
     ws = torch.empty(max(16, pa.pf_cfg_workspace_bytes(wl.batch, n)), dtype=torch.uint8, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    # flush by reading 512 MB (a read leaves clean lines, so the timed call pays no write-backs)
+    flush = torch.ones(128 << 20, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     times = []
     for i in range(reps + 3):
-        flush.zero_()
+        flush.sum()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         pa.pf_cfg_combine_relmae(c, u, wl.w, out_f, out_b, rel, ws)
@@ -526,8 +527,46 @@ def run_e2e(args, world, local, wl, sets, pat, outs, c_in, u_in, cfg_out, rel, w
             "d2h_bytes_per_step": d2h, "copies": "pinned host, overlapped per patch on two copy streams"}
 
 
+def run_profile_calls(args):
+    """For ncu captures: the start-up pass and `n` micro-steps (patches 0..n-1) of one layer of
+    the workload, nothing else.  Small device footprint (one layer)."""
+    import patch_attention_b200 as pa
+
+    wl0 = synth.ATTN_WORKLOADS[args.workload]
+    wl = synth.AttnWorkload(wl0.name, wl0.batch, wl0.heads, wl0.head_dim, wl0.grid_h, wl0.grid_w,
+                            wl0.n_patches, wl0.n_txt, 1, 2, wl0.ar_a, wl0.ar_b, wl0.qk_rmsnorm)
+    t = synth.AttnInputs(wl, device="cuda").step_tensors(0)
+    pat = pa.PatchAttention(wl.batch, wl.heads, wl.head_dim, wl.n_img, wl.n_patches, wl.n_txt, 1)
+    pat.init_layer(0, t["k"], t["v"])
+    P = wl.patch_len
+    for p in range(min(args.profile_calls, wl.n_patches)):
+        sl = slice(p * P, (p + 1) * P)
+        pat.step(0, p, t["q"][:, sl].contiguous(), t["k"][:, sl].contiguous(),
+                 t["v"][:, sl].contiguous(), t["k_txt"], t["v_txt"])
+    torch.cuda.synchronize()
+    pat.check()
+    pat.close()
+    return 0
+
+
+def run_profile_cfg(args):
+    """For ncu captures: two guidance-kernel calls at the largest sweep size."""
+    import patch_attention_b200 as pa
+
+    wl = synth.CfgWorkload("cfg", 4, 16, 512, 512)
+    c, u = synth.CfgInputs(wl, device="cuda").step_tensors(25)
+    for _ in range(2):
+        pa.cfg_combine_relmae(c, u, wl.w)
+    torch.cuda.synchronize()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--profile-calls", type=int, default=0,
+                    help="only run the start-up pass and this many micro-steps of one layer (for ncu)")
+    ap.add_argument("--profile-cfg", action="store_true",
+                    help="only run two guidance-kernel calls at the largest size (for ncu)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
@@ -539,6 +578,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3 and args.impl != "reference":
         args.warmup = 3
+    if args.profile_calls > 0:
+        return run_profile_calls(args)
+    if args.profile_cfg:
+        return run_profile_cfg(args)
     world, rank, local = dist_setup()
     try:
         if args.impl == "reference":

@@ -43,6 +43,8 @@ __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
 __global__ void __launch_bounds__(kThreads) cfg_partial_kernel(
     const float4* __restrict__ c, const float4* __restrict__ u, int64_t n4, float w,
     float4* __restrict__ out_f32, uint2* __restrict__ out_bf16, double2* __restrict__ partials) {
+  // let the finalize kernel be scheduled now; it waits for this grid's completion itself
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int b = blockIdx.y;
   const int g = blockIdx.x;
   const int G = gridDim.x;
@@ -109,6 +111,9 @@ __global__ void __launch_bounds__(kThreads) cfg_partial_kernel(
 
 __global__ void cfg_finalize_kernel(const double2* __restrict__ partials, int G,
                                     float* __restrict__ relmae) {
+  // launched as a programmatic dependent of cfg_partial_kernel: wait until that grid has
+  // finished and its partials are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.x;
   const int lane = threadIdx.x;
   double num = 0.0, den = 0.0;
@@ -150,8 +155,20 @@ cudaError_t launch_cfg_combine_relmae(const float* c, const float* u, int batch,
       reinterpret_cast<double2*>(workspace));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  cfg_finalize_kernel<<<batch, 32, 0, stream>>>(reinterpret_cast<const double2*>(workspace), G, relmae);
-  return cudaGetLastError();
+  // programmatic dependent launch: the finalize is scheduled while the partial kernel runs
+  // (hiding its launch latency) and synchronises on it with griddepcontrol.wait
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(batch);
+  cfg.blockDim = dim3(32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, cfg_finalize_kernel, reinterpret_cast<const double2*>(workspace), G,
+                            relmae);
 }
 
 }  // namespace pf
