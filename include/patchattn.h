@@ -152,6 +152,27 @@ pf_status pf_cfg_combine_relmae(const float* eps_c, const float* eps_u, int batc
                                 uint16_t* out_bf16, float* relmae, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
+/* Same computation and outputs as pf_cfg_combine_relmae, for callers that cannot allocate
+ * device memory: code that runs where another framework owns the device allocator and must
+ * see every allocation, loops that cannot afford the device synchronisation a cudaMalloc may
+ * imply, or host callbacks that may not make allocation calls.  The pages have no
+ * counterpart of this entry point; it is a deployment convenience.
+ *
+ * The partial sums go to a fixed 64 KiB array inside the library's device image (4096
+ * partial-sum pairs) instead of a caller workspace, so the call allocates nothing and takes
+ * no workspace argument.  Limit: batch <= 4096 samples; a larger batch returns PF_ERR_SHAPE.
+ * Every GPU that loads the library holds the array until the process exits.
+ *
+ * Set-up: the first call on each device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream capture.
+ * The array is shared by all calls and keeps the last call's contents; nothing in it needs
+ * to start at zero (each call writes every slot it reads).  Calls whose work overlaps on the
+ * GPU (different streams, or different host threads) race on the array: serialise them.
+ * Errors as for pf_cfg_combine_relmae; PF_ERR_CUDA if the address lookup fails. */
+pf_status pf_cfg_combine_relmae_static(const float* eps_c, const float* eps_u, int batch,
+                                       int64_t n_per_sample, float w, float* out_f32,
+                                       uint16_t* out_bf16, float* relmae, void* stream);
+
 /* Synchronise `stream`, then read the device status word the context's kernels write when
  * a bounded wait expires: PF_ERR_TIMEOUT if any did (and clear it), PF_ERR_CUDA if the
  * stream reported an error, else PF_OK. */

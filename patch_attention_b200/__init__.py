@@ -35,7 +35,7 @@ PF_SCHED_DISTRIFUSION = 1
 EXPORTED = [
     "pf_kvbuf_bytes", "pf_create", "pf_destroy", "pf_kvbuf_init", "pf_patch_attn_step",
     "pf_get_state", "pf_set_state", "pf_workspace_bytes", "pf_set_workspace",
-    "pf_cfg_workspace_bytes", "pf_cfg_combine_relmae",
+    "pf_cfg_workspace_bytes", "pf_cfg_combine_relmae", "pf_cfg_combine_relmae_static",
     "pf_check_device_status", "pf_status_string", "pf_version",
 ]
 
@@ -78,6 +78,7 @@ def _lib():
             "pf_set_state": (i, [vp, i, i]),
             "pf_cfg_workspace_bytes": (sz, [i, i64]),
             "pf_cfg_combine_relmae": (i, [vp, vp, i, i64, f, vp, vp, vp, vp, sz, vp]),
+            "pf_cfg_combine_relmae_static": (i, [vp, vp, i, i64, f, vp, vp, vp, vp]),
             "pf_check_device_status": (i, [vp, vp]),
             "pf_status_string": (ctypes.c_char_p, [i]),
             "pf_version": (i, []),
@@ -209,6 +210,23 @@ def pf_cfg_combine_relmae(eps_c: torch.Tensor, eps_u: torch.Tensor, w: float,
     ws = _ptr(workspace, torch.uint8, None, "workspace")
     _check(_lib().pf_cfg_combine_relmae(c, u, B, n, float(w), of, ob, r, ws, workspace.numel(),
                                         _stream(stream)), "pf_cfg_combine_relmae")
+
+
+def pf_cfg_combine_relmae_static(eps_c: torch.Tensor, eps_u: torch.Tensor, w: float,
+                                 out_f32: Optional[torch.Tensor], out_bf16: Optional[torch.Tensor],
+                                 relmae: torch.Tensor, stream=None) -> None:
+    """The guidance combine without a workspace argument: the library keeps its partial sums
+    in a fixed device array, so nothing is allocated for the call (batch <= 4096).  Calls
+    that run concurrently on the GPU share that array and must not overlap."""
+    B = eps_c.shape[0]
+    n = eps_c.numel() // B
+    c = _ptr(eps_c, torch.float32, None, "eps_c")
+    u = _ptr(eps_u, torch.float32, tuple(eps_c.shape), "eps_u")
+    of = _ptr(out_f32, torch.float32, tuple(eps_c.shape), "out_f32")
+    ob = _ptr(out_bf16, torch.bfloat16, tuple(eps_c.shape), "out_bf16")
+    r = _ptr(relmae, torch.float32, (B,), "relmae")
+    _check(_lib().pf_cfg_combine_relmae_static(c, u, B, n, float(w), of, ob, r, _stream(stream)),
+           "pf_cfg_combine_relmae_static")
 
 
 def pf_check_device_status(ctx, stream=None) -> None:

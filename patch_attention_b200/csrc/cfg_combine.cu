@@ -13,6 +13,8 @@
 
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "pf_internal.h"
 
 namespace pf {
@@ -138,6 +140,52 @@ __global__ void cfg_finalize_kernel(const double2* __restrict__ partials, int G,
 }
 
 }  // namespace
+
+// ----------------------------------------------------------------------------------------
+// Variant with no caller workspace: the fp64 partial sums go to a fixed array that lives in
+// this library's device image, so the call needs no device allocation at all.
+
+// 4096 partial-sum pairs (64 KiB).  One pair per (sample, block) of the partial kernel; the
+// grid gives a batch of B samples at most max(B, 1184) pairs, so any batch up to 4096 fits.
+constexpr int kStaticPartials = 4096;
+static __device__ __align__(256) double2 g_cfg_static_partials[kStaticPartials];
+
+namespace {
+// Device address of g_cfg_static_partials per device ordinal.  In host code the array's name
+// only stands in for the symbol; the address must be asked of the runtime with the device
+// current, once per device.
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_addr[kMaxDevices] = {};
+}  // namespace
+
+int cfg_static_capacity_samples() { return kStaticPartials; }
+
+cudaError_t launch_cfg_combine_relmae_static(const float* c, const float* u, int batch, int64_t n,
+                                             float w, float* out_f32, uint16_t* out_bf16,
+                                             float* relmae, cudaStream_t stream) {
+  const int G = blocks_per_sample(batch, n);
+  if (static_cast<int64_t>(batch) * G > kStaticPartials) return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (g_static_addr[dev] == nullptr) {
+      e = cudaGetSymbolAddress(&g_static_addr[dev], g_cfg_static_partials);
+      if (e != cudaSuccess) {
+        g_static_addr[dev] = nullptr;
+        return e;
+      }
+    }
+    scratch = g_static_addr[dev];
+  }
+  // Every slot the finalize reads is written by the partial kernel of the same call, so the
+  // array needs no clearing between calls.
+  return launch_cfg_combine_relmae(c, u, batch, n, w, out_f32, out_bf16, relmae, scratch, stream);
+}
 
 size_t cfg_workspace_bytes(int batch, int64_t n_per_sample) {
   if (batch < 1 || n_per_sample < 4) return 0;

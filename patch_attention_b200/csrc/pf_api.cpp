@@ -343,6 +343,24 @@ pf_status pf_cfg_combine_relmae(const float* eps_c, const float* eps_u, int batc
                                                  static_cast<cudaStream_t>(stream)));
 }
 
+pf_status pf_cfg_combine_relmae_static(const float* eps_c, const float* eps_u, int batch,
+                                       int64_t n_per_sample, float w, float* out_f32,
+                                       uint16_t* out_bf16, float* relmae, void* stream) {
+  if (!eps_c || !eps_u || !relmae) return PF_ERR_INVALID_ARG;
+  if (batch < 1 || n_per_sample < 4) return PF_ERR_SHAPE;
+  if (n_per_sample % 4 != 0) return PF_ERR_SHAPE;
+  if (batch > pf::cfg_static_capacity_samples()) return PF_ERR_SHAPE;
+  if (static_cast<double>(batch) * static_cast<double>(n_per_sample) > 9.0e15) return PF_ERR_SHAPE;
+  if (!std::isfinite(w)) return PF_ERR_INVALID_ARG;
+  if (!aligned16(eps_c) || !aligned16(eps_u) || (out_f32 && !aligned16(out_f32)) ||
+      (out_bf16 && (reinterpret_cast<uintptr_t>(out_bf16) & 7u)) ||
+      (reinterpret_cast<uintptr_t>(relmae) & 3u))
+    return PF_ERR_ALIGN;
+  return from_cuda(pf::launch_cfg_combine_relmae_static(eps_c, eps_u, batch, n_per_sample, w, out_f32,
+                                                        out_bf16, relmae,
+                                                        static_cast<cudaStream_t>(stream)));
+}
+
 pf_status pf_check_device_status(pf_ctx* ctx, void* stream) {
   if (!ctx) return PF_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PF_ERR_CUDA;

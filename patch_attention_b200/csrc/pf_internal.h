@@ -61,6 +61,13 @@ cudaError_t launch_cfg_combine_relmae(const float* c, const float* u, int batch,
                                       float w, float* out_f32, uint16_t* out_bf16, float* relmae,
                                       void* workspace, cudaStream_t stream);
 
+// Guidance combine + rel-MAE with its partial sums in a static device array of the library
+// (no caller workspace).  Returns cudaErrorInvalidValue if the batch exceeds the array.
+cudaError_t launch_cfg_combine_relmae_static(const float* c, const float* u, int batch, int64_t n,
+                                             float w, float* out_f32, uint16_t* out_bf16,
+                                             float* relmae, cudaStream_t stream);
+int cfg_static_capacity_samples();
+
 // Device word written by kernels whose bounded waits expired (0 = none).
 cudaError_t read_and_clear_watchdog(unsigned* value);
 
