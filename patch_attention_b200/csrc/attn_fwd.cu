@@ -214,8 +214,11 @@ __device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) {
                fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
 }
 
-// p_k = 2^(s_k c - m) with the special-function unit, packed to bf16 pairs; returns the
-// fp32 sum.  Masked keys (-inf) give exactly 0.
+// p_k = 2^(s_k c - m), packed to bf16 pairs; returns the fp32 sum.  POLY of every 8 pairs
+// of columns use the FMA-pipe polynomial, the rest the special-function unit.  With
+// POLY = 0, masked keys (-inf) give exactly 0 (the polynomial clamps, so masked tiles must
+// use POLY = 0).
+template <int POLY = 0>
 __device__ __forceinline__ void exact_exps(const uint32_t (&s)[128], float c, float m,
                                            uint32_t (&pk)[64], float& lsum) {
   const float2 cc = make_float2(c, c), nm = make_float2(-m, -m);
@@ -224,7 +227,7 @@ __device__ __forceinline__ void exact_exps(const uint32_t (&s)[128], float c, fl
 #pragma unroll
   for (int k = 0; k < 64; ++k) {
     const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), cc, nm);
-    const float2 p = make_float2(ex2(x.x), ex2(x.y));
+    const float2 p = (k & 7) < POLY ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
     acc[k & 3] = __fadd2_rn(acc[k & 3], p);
     pk[k] = pack_bf16(p.x, p.y);
   }
@@ -261,10 +264,11 @@ __device__ __forceinline__ float speculative_exps(const uint32_t (&s)[128], floa
 }
 
 // Of every 8 pairs of columns, the pairs whose exponentials run on the FMA pipe instead of
-// the special-function unit (3/8: balances the unit's 16 results/clk/SM against the extra
-// issue slots of the polynomial, about 5 instructions per element).
+// the special-function unit.  The polynomial costs about 5 issue slots per element against
+// 1 for the unit (16 results/clk/SM); measured over 0..4 of 8, 2 of 8 was fastest for both
+// head_dim 64 and 128.
 template <int D>
-constexpr int kPolyPairs = 3;
+constexpr int kPolyPairs = 2;
 
 __device__ __forceinline__ void raise_abort(volatile int* abort, unsigned code) {
   *abort = 1;
@@ -275,6 +279,9 @@ template <int D, int NQ>
 __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_constant__ AttnParams p) {
   using Dm = Dims<D>;
   constexpr int S = Dm::kStages;
+  // head_dim 64: O_t needs only 64 of its 128 TMEM columns, so P_t lives in the other 64
+  // instead of over S_t, and the next QK need not wait for the current PV.
+  constexpr bool kSepP = Dm::kMmaN <= 64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -288,7 +295,9 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
   uint64_t* p_full = s_full + 2;
   uint64_t* o_full = p_full + 2;
   uint64_t* mma_done = o_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* s_free = mma_done + 1;   // separate-P layout: softmax has S in registers
+  uint64_t* pv_done = s_free + 2;    // separate-P layout: PV of a tile has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -313,6 +322,10 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
       mbar_init(smem_u32(o_full + t), 1);
     }
     mbar_init(smem_u32(mma_done), 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(smem_u32(s_free + t), 4);  // one arrival per softmax warp
+      mbar_init(smem_u32(pv_done + t), 1);
+    }
     *abort = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -395,32 +408,76 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
       const uint32_t q_base = smem_u32(sQ);
       const uint32_t kv_base = smem_u32(sKV);
 
-      // Base descriptors are built once; an operand at byte offset `off` from a base only
-      // changes the 14-bit start-address field, by off >> 4 (no carry: smem < 256 KB).
-      const uint64_t dq0 = smem_desc_sw128(q_base, 16, 1024);
-      const uint64_t dk0 = smem_desc_sw128(kv_base, 16, 1024);
-      const uint64_t dv0 = smem_desc_sw128(kv_base, kChunkBytes, 1024);
-      auto issue_qk = [&](int t, int st) {
-        const uint64_t a0 = dq0 + static_cast<uint64_t>((t * Dm::kTileBytes) >> 4);
-        const uint64_t b0 = dk0 + static_cast<uint64_t>((st * Dm::kTileBytes) >> 4);
+      // Descriptor low words (start address >> 4 | LBO) of the operand bases; an operand at
+      // byte offset `off` from a base only adds off >> 4 to the 14-bit start-address field
+      // (no carry: shared memory < 256 KB).  The high word is a compile-time constant.
+      const uint32_t q_lo = (q_base >> 4) | desc_lbo_bits(16);
+      const uint32_t k_lo = (kv_base >> 4) | desc_lbo_bits(16);
+      const uint32_t v_lo = (kv_base >> 4) | desc_lbo_bits(kChunkBytes);
+      auto issue_qk = [=](int t, int st) {
+        const uint32_t a0 = q_lo + static_cast<uint32_t>((t * Dm::kTileBytes) >> 4);
+        const uint32_t b0 = k_lo + static_cast<uint32_t>((st * Dm::kTileBytes) >> 4);
         const uint32_t d = tmem + t * 128;
 #pragma unroll
         for (int kk = 0; kk < Dm::kMmaN / 16; ++kk) {
-          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
-          mma_ss(d, a0 + off, b0 + off, idesc_qk, kk > 0);
+          const uint32_t off = static_cast<uint32_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+          mma_ss(d, smem_desc_lo(a0 + off), smem_desc_lo(b0 + off), idesc_qk, kk > 0);
         }
       };
-      auto issue_pv = [&](int t, int st, bool acc) {
-        const uint64_t v0 = dv0 + static_cast<uint64_t>((st * Dm::kTileBytes) >> 4);
+      auto issue_pv = [=](int t, int st, bool acc) {
+        const uint32_t v0 = v_lo + static_cast<uint32_t>((st * Dm::kTileBytes) >> 4);
         const uint32_t d = tmem + kColO + t * 128;
-        const uint32_t a = tmem + t * 128;
+        const uint32_t a = tmem + (kSepP ? kColO + t * 128 + 64 : t * 128);
 #pragma unroll
         for (int kk = 0; kk < kRows / 16; ++kk)
-          mma_ts(d, a + kk * 8, v0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv, acc || kk > 0);
+          mma_ts(d, a + kk * 8, smem_desc_lo(v0 + static_cast<uint32_t>((kk * 2048) >> 4)), idesc_pv,
+                 acc || kk > 0);
       };
 
       bool ok = mbar_wait(smem_u32(q_full), 0, abort, kWaitNs);
       tc_fence_after();
+      if constexpr (kSepP) {
+        // P has its own TMEM columns: QK of the next key tile is issued as soon as the
+        // softmax has S of the current one in registers, so the tensor core computes
+        // S(j+1) while the softmax is still exponentiating tile j.
+        if (ok && n_tiles > 0) {
+          ok = mbar_wait(smem_u32(kv_full + 0), 0, abort, kWaitNs);  // K(0): load 0, stage 0
+          tc_fence_after();
+          if (ok) {
+            for (int t = 0; t < NQ; ++t) {
+              issue_qk(t, 0);
+              mma_commit(smem_u32(s_full + t));
+            }
+            mma_commit(smem_u32(kv_empty + 0));
+          }
+        }
+        for (int j = 0; j < n_tiles && ok; ++j) {
+          if (j + 1 < n_tiles) {
+            const int iK = 2 * (j + 1), sK = iK % S;
+            if (!(ok = mbar_wait(smem_u32(kv_full + sK), (iK / S) & 1, abort, kWaitNs))) break;
+            tc_fence_after();
+            for (int t = 0; t < NQ; ++t) {
+              if (!(ok = mbar_wait(smem_u32(s_free + t), j & 1, abort, kWaitNs))) break;
+              tc_fence_after();
+              issue_qk(t, sK);
+              mma_commit(smem_u32(s_full + t));
+            }
+            if (!ok) break;
+            mma_commit(smem_u32(kv_empty + sK));
+          }
+          const int iV = 2 * j + 1, sV = iV % S;
+          if (!(ok = mbar_wait(smem_u32(kv_full + sV), (iV / S) & 1, abort, kWaitNs))) break;
+          tc_fence_after();
+          for (int t = 0; t < NQ; ++t) {
+            if (!(ok = mbar_wait(smem_u32(p_full + t), j & 1, abort, kWaitNs))) break;
+            tc_fence_after();
+            issue_pv(t, sV, j > 0);
+            mma_commit(smem_u32(pv_done + t));
+          }
+          if (!ok) break;
+          mma_commit(smem_u32(kv_empty + sV));
+        }
+      } else {
       for (int j = 0; j < n_tiles && ok; ++j) {
         const int iK = 2 * j, sK = iK % S;
         if (!(ok = mbar_wait(smem_u32(kv_full + sK), (iK / S) & 1, abort, kWaitNs))) break;
@@ -460,6 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
           mma_commit(smem_u32(o_full + t));
         }
         if (ok) mma_commit(smem_u32(kv_empty + sV));
+      }
       }
       if (!ok) raise_abort(abort, kWdMma);
       // drain every MMA issued by this thread before TMEM is released
@@ -534,6 +592,62 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
       const int nv = seg.nvalid(j0 + j);
       uint32_t pk[64];
       float lsum;
+      if constexpr (kSepP) {
+        // S is in registers: hand its TMEM columns back so QK of the next tile can start.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(s_free + t));
+        if (nv < kRows) {
+#pragma unroll
+          for (int k = 0; k < 128; ++k)
+            if (k >= nv) s[k] = __float_as_uint(-INFINITY);
+        }
+        const float mxs = row_max128(s) * c;
+        bool pv_seen = (j == 0);  // PV of the previous tile done: O stable, P columns free
+        if (mxs > m + 8.f) {
+          const float alpha = ex2(m - mxs);
+          l *= alpha;
+          if (j > 0) {
+            ok = mbar_wait(smem_u32(pv_done + t), (j - 1) & 1, abort, kWaitNs);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            pv_seen = true;
+#pragma unroll
+            for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
+              uint32_t o[16];
+              tmem_ld16(tO + c0, o);
+              tmem_wait_ld();
+              reg_fence<16>(o);
+#pragma unroll
+              for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+              tmem_st16(tO + c0, o);
+            }
+          }
+          m = mxs;
+        }
+        if (nv < kRows)
+          exact_exps<0>(s, c, m, pk, lsum);
+        else
+          exact_exps<kPolyPairs<D>>(s, c, m, pk, lsum);
+        l += lsum;
+        if (!pv_seen) {
+          ok = mbar_wait(smem_u32(pv_done + t), (j - 1) & 1, abort, kWaitNs);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        if (wq == 0 && lane == 0) PF_TRACE_AT(7, t, j);
+        tmem_st32(tO + 64, pk);
+        tmem_st32(tO + 96, pk + 32);
+        tmem_wait_st();
+        if (wq == 0 && lane == 0) PF_TRACE_AT(8, t, j);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(p_full + t));
+        if (wq == 0 && lane == 0) PF_TRACE_AT(1, t, j);
+        continue;
+      }
       // Fast path: exponentiate against the current reference maximum m straight away and
       // check afterwards that no value exceeded 2^8; the row maximum is then off the
       // critical path.  The first tile (no reference yet), ragged tiles (masked keys) and
@@ -591,7 +705,9 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
     }
     if (!ok && lane == 0) raise_abort(abort, kWdSoftmax);
     {
-      bool ok_o = ok && mbar_wait(smem_u32(o_full + t), 0, abort, kWaitNs);
+      // final O: the last PV of this tile (separate-P layout) or the o_full commit
+      bool ok_o = ok && (kSepP ? mbar_wait(smem_u32(pv_done + t), (n_tiles - 1) & 1, abort, kWaitNs)
+                               : mbar_wait(smem_u32(o_full + t), 0, abort, kWaitNs));
       ok_o = __all_sync(0xffffffffu, ok_o);
       // the whole warpgroup takes the same branch (the merge path has barriers)
       ok_o = named_bar_and(1 + t, kRows, ok_o);

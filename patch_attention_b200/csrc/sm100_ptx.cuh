@@ -238,6 +238,17 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t start, uint32_t lbo
   return d;
 }
 
+// The same descriptor split in halves for a fixed SBO of 1024 bytes: the high word
+// (SBO, version, layout) is a compile-time constant, the low word carries the start
+// address and the LBO.  Building a descriptor is then one 32-bit OR per MMA.
+constexpr uint32_t kDescHiSw128Sbo1024 = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint64_t smem_desc_lo(uint32_t lo) {
+  return (static_cast<uint64_t>(kDescHiSw128Sbo1024) << 32) | lo;
+}
+__host__ __device__ constexpr uint32_t desc_lbo_bits(uint32_t lbo_bytes) {
+  return ((lbo_bytes >> 4) & 0x3FFFu) << 16;
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
 //   b_mn_major: 0 = B is K-major, 1 = B is MN-major
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, int b_mn_major) {
