@@ -173,6 +173,39 @@ pf_status pf_cfg_combine_relmae_static(const float* eps_c, const float* eps_u, i
                                        int64_t n_per_sample, float w, float* out_f32,
                                        uint16_t* out_bf16, float* relmae, void* stream);
 
+/* Hybrid-CFG adaptive switching ("조건부 가이드 스케줄링 기반 하이브리드 데이터-파이프라인 병렬 처리를
+ * 통한 디퓨전 모델 가속화", second block 단락 2-3): the denoising steps are divided into
+ * Warm-Up, Parallelism and Fully-Connecting; the switch points tau1 and tau2 follow rel-MAE_t,
+ * and parallelism is active while rel-MAE_t has settled below a threshold.  The pages give
+ * no threshold values, so they are parameters:
+ *   - Warm-Up -> Parallelism (tau1) once rel-MAE_t <= enter_below for enter_patience
+ *     consecutive steps;
+ *   - Parallelism -> Fully-Connecting (tau2) once rel-MAE_t >= exit_above, or after
+ *     max_parallel_steps parallel steps (<= 0: no limit).  Fully-Connecting is final.
+ * Host-only state, no allocation; one pf_switch per image (rel-MAE_t is per sample). */
+typedef enum { PF_PHASE_WARMUP = 0, PF_PHASE_PARALLEL = 1, PF_PHASE_FULL = 2 } pf_phase;
+
+typedef struct {
+  float enter_below;
+  int enter_patience;
+  float exit_above;
+  int max_parallel_steps;
+  int phase;          /* pf_phase that applies to the next step */
+  int step;           /* steps observed so far */
+  int below_run;      /* consecutive steps with rel-MAE_t <= enter_below */
+  int parallel_steps; /* steps spent in Parallelism */
+  int tau1, tau2;     /* step indices where the phase changed (-1 until then) */
+} pf_switch;
+
+/* Initialise a controller (phase Warm-Up).  PF_ERR_INVALID_ARG for NULL, a non-finite or
+ * negative threshold, or enter_patience < 1. */
+pf_status pf_switch_init(pf_switch* s, float enter_below, int enter_patience, float exit_above,
+                         int max_parallel_steps);
+
+/* Feed rel-MAE_t of the step just finished; *phase_out (may be NULL) receives the phase for
+ * the next step.  NaN rel-MAE_t is rejected with PF_ERR_INVALID_ARG and leaves the state. */
+pf_status pf_switch_update(pf_switch* s, float relmae, int* phase_out);
+
 /* Synchronise `stream`, then read the device status word the context's kernels write when
  * a bounded wait expires: PF_ERR_TIMEOUT if any did (and clear it), PF_ERR_CUDA if the
  * stream reported an error, else PF_OK. */

@@ -21,6 +21,7 @@ from .attention import (  # noqa: F401
     image_key_rows,
     patch_keys,
     patch_attention,
+    distrifusion_attention,
     expected_buffer,
     KVBufferWalk,
 )

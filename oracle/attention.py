@@ -79,6 +79,27 @@ def patch_attention(q_now, k_now, v_now, k_prev, v_prev, k_txt, v_txt, p, n_patc
     return attend(q, k, v, scale)
 
 
+def distrifusion_attention(q_now, k_now, v_now, k_prev, v_prev, k_txt, v_txt, p, n_patches,
+                           scale, rows=None):
+    """Output rows of patch p under the DistriFusion schedule.
+
+    "기술 요약: PipeFusion", 문제 정의 (DistriFusion): every device keeps the full-spatial K/V of
+    every layer and works from the previous step's activations; 주요 기여 / 품질 보존: it relies
+    on stale data more than PipeFusion.  Reading used here: patch p sees its own rows at this
+    step and every other image row at the previous step, whatever order the patches run in.
+    """
+    plen = q_now.shape[0] // n_patches
+    idx = np.arange(plen) if rows is None else np.asarray(rows)
+    own = np.zeros(k_now.shape[0], dtype=bool)
+    own[p * plen:(p + 1) * plen] = True
+    shape = (k_now.shape[0],) + (1,) * (k_now.ndim - 1)
+    k_img = np.where(own.reshape(shape), k_now, k_prev)
+    v_img = np.where(own.reshape(shape), v_now, v_prev)
+    q = q_now[p * plen + idx]
+    return attend(q, np.concatenate([k_img, k_txt], axis=0), np.concatenate([v_img, v_txt], axis=0),
+                  scale)
+
+
 def expected_buffer(x_now, x_prev, p, n_patches):
     """Contents of a layer's KV buffer after the call for patch p (image rows only)."""
     return image_key_rows(x_now, x_prev, p, n_patches)

@@ -36,8 +36,13 @@ EXPORTED = [
     "pf_kvbuf_bytes", "pf_create", "pf_destroy", "pf_kvbuf_init", "pf_patch_attn_step",
     "pf_get_state", "pf_set_state", "pf_workspace_bytes", "pf_set_workspace",
     "pf_cfg_workspace_bytes", "pf_cfg_combine_relmae", "pf_cfg_combine_relmae_static",
-    "pf_check_device_status", "pf_status_string", "pf_version",
+    "pf_check_device_status", "pf_status_string", "pf_version", "pf_switch_init",
+    "pf_switch_update",
 ]
+
+PF_PHASE_WARMUP = 0
+PF_PHASE_PARALLEL = 1
+PF_PHASE_FULL = 2
 
 
 class pf_config(ctypes.Structure):
@@ -45,6 +50,15 @@ class pf_config(ctypes.Structure):
         ("batch", ctypes.c_int), ("heads", ctypes.c_int), ("head_dim", ctypes.c_int),
         ("n_img", ctypes.c_int), ("n_patches", ctypes.c_int), ("n_txt", ctypes.c_int),
         ("n_layers", ctypes.c_int), ("softmax_scale", ctypes.c_float), ("schedule", ctypes.c_int),
+    ]
+
+
+class pf_switch(ctypes.Structure):
+    _fields_ = [
+        ("enter_below", ctypes.c_float), ("enter_patience", ctypes.c_int),
+        ("exit_above", ctypes.c_float), ("max_parallel_steps", ctypes.c_int),
+        ("phase", ctypes.c_int), ("step", ctypes.c_int), ("below_run", ctypes.c_int),
+        ("parallel_steps", ctypes.c_int), ("tau1", ctypes.c_int), ("tau2", ctypes.c_int),
     ]
 
 
@@ -81,6 +95,8 @@ def _lib():
             "pf_cfg_combine_relmae_static": (i, [vp, vp, i, i64, f, vp, vp, vp, vp]),
             "pf_check_device_status": (i, [vp, vp]),
             "pf_status_string": (ctypes.c_char_p, [i]),
+            "pf_switch_init": (i, [ctypes.POINTER(pf_switch), f, i, f, i]),
+            "pf_switch_update": (i, [ctypes.POINTER(pf_switch), f, ctypes.POINTER(i)]),
             "pf_version": (i, []),
         }
         for name, (res, args) in sig.items():
@@ -227,6 +243,31 @@ def pf_cfg_combine_relmae_static(eps_c: torch.Tensor, eps_u: torch.Tensor, w: fl
     r = _ptr(relmae, torch.float32, (B,), "relmae")
     _check(_lib().pf_cfg_combine_relmae_static(c, u, B, n, float(w), of, ob, r, _stream(stream)),
            "pf_cfg_combine_relmae_static")
+
+
+class HybridCfgSwitch:
+    """Warm-Up -> Parallelism -> Fully-Connecting controller driven by rel-MAE_t (one per
+    image); see pf_switch_init in include/patchattn.h for the rule and its parameters."""
+
+    def __init__(self, enter_below: float, enter_patience: int = 1, exit_above: float = float("inf"),
+                 max_parallel_steps: int = 0):
+        self.state = pf_switch()
+        _check(_lib().pf_switch_init(ctypes.byref(self.state), enter_below, enter_patience,
+                                     exit_above, max_parallel_steps), "pf_switch_init")
+
+    def update(self, relmae: float) -> int:
+        ph = ctypes.c_int()
+        _check(_lib().pf_switch_update(ctypes.byref(self.state), float(relmae), ctypes.byref(ph)),
+               "pf_switch_update")
+        return ph.value
+
+    @property
+    def phase(self) -> int:
+        return self.state.phase
+
+    @property
+    def tau(self):
+        return self.state.tau1, self.state.tau2
 
 
 def pf_check_device_status(ctx, stream=None) -> None:

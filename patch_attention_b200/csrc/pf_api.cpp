@@ -361,6 +361,50 @@ pf_status pf_cfg_combine_relmae_static(const float* eps_c, const float* eps_u, i
                                                         static_cast<cudaStream_t>(stream)));
 }
 
+pf_status pf_switch_init(pf_switch* s, float enter_below, int enter_patience, float exit_above,
+                         int max_parallel_steps) {
+  if (!s || !std::isfinite(enter_below) || enter_below < 0.f || std::isnan(exit_above) ||
+      exit_above < 0.f || enter_patience < 1)
+    return PF_ERR_INVALID_ARG;
+  s->enter_below = enter_below;
+  s->enter_patience = enter_patience;
+  s->exit_above = exit_above;
+  s->max_parallel_steps = max_parallel_steps;
+  s->phase = PF_PHASE_WARMUP;
+  s->step = 0;
+  s->below_run = 0;
+  s->parallel_steps = 0;
+  s->tau1 = -1;
+  s->tau2 = -1;
+  return PF_OK;
+}
+
+pf_status pf_switch_update(pf_switch* s, float relmae, int* phase_out) {
+  if (!s || std::isnan(relmae)) return PF_ERR_INVALID_ARG;
+  const int t = s->step++;
+  switch (s->phase) {
+    case PF_PHASE_WARMUP:
+      s->below_run = relmae <= s->enter_below ? s->below_run + 1 : 0;
+      if (s->below_run >= s->enter_patience) {
+        s->phase = PF_PHASE_PARALLEL;
+        s->tau1 = t + 1;
+      }
+      break;
+    case PF_PHASE_PARALLEL:
+      ++s->parallel_steps;
+      if (relmae >= s->exit_above ||
+          (s->max_parallel_steps > 0 && s->parallel_steps >= s->max_parallel_steps)) {
+        s->phase = PF_PHASE_FULL;
+        s->tau2 = t + 1;
+      }
+      break;
+    default:
+      break;
+  }
+  if (phase_out) *phase_out = s->phase;
+  return PF_OK;
+}
+
 pf_status pf_check_device_status(pf_ctx* ctx, void* stream) {
   if (!ctx) return PF_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PF_ERR_CUDA;

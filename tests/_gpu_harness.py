@@ -133,6 +133,13 @@ def run_workload(wl: synth.AttnWorkload, steps: Optional[int] = None, full_check
                             vmax = _vmax(cur_cpu, prev_cpu, p, wl.n_patches, bi, slice(h, h + 1), schedule)
                             got = f64(o[bi][rows][:, h:h + 1])
                             chk.add(got, ref, vmax, f"s{s} l{layer} p{p} b{bi} h{h} rows")
+                if schedule == pa.PF_SCHED_DISTRIFUSION:
+                    # after the step, one half of the buffer holds exactly this step's K/V
+                    # (the stale context of the next step)
+                    halves = [pat.buffer_kv(layer, hf) for hf in (0, 1)]
+                    assert any(torch.equal(kb.view(torch.int16), cur["k"].view(torch.int16)) and
+                               torch.equal(vb.view(torch.int16), cur["v"].view(torch.int16))
+                               for kb, vb in halves), "no buffer half holds the step's K/V"
                 prev[layer] = cur
             pat.check()
         torch.cuda.synchronize()
@@ -144,19 +151,12 @@ def run_workload(wl: synth.AttnWorkload, steps: Optional[int] = None, full_check
 def _ref(wl, cur_cpu, prev_cpu, p, b, rows, heads, schedule):
     if schedule == pa.PF_SCHED_PIPEFUSION:
         return oracle_patch_output(wl, cur_cpu, prev_cpu, p, b, rows, heads)
-    # DistriFusion: only the patch's own rows are this step's; everything else stale
     sl = slice(None) if heads is None else heads
     take = lambda t: f64(t[b][:, sl])
-    P = wl.patch_len
-    k = take(prev_cpu["k"]).copy()
-    v = take(prev_cpu["v"]).copy()
-    k[p * P:(p + 1) * P] = take(cur_cpu["k"])[p * P:(p + 1) * P]
-    v[p * P:(p + 1) * P] = take(cur_cpu["v"])[p * P:(p + 1) * P]
-    q = take(cur_cpu["q"])[p * P:(p + 1) * P]
-    if rows is not None:
-        q = q[rows]
-    return oracle.attend(q, np.concatenate([k, take(cur_cpu["k_txt"])]),
-                         np.concatenate([v, take(cur_cpu["v_txt"])]), wl.softmax_scale)
+    return oracle.distrifusion_attention(
+        take(cur_cpu["q"]), take(cur_cpu["k"]), take(cur_cpu["v"]), take(prev_cpu["k"]),
+        take(prev_cpu["v"]), take(cur_cpu["k_txt"]), take(cur_cpu["v_txt"]), p, wl.n_patches,
+        wl.softmax_scale, rows=rows)
 
 
 def _vmax(cur_cpu, prev_cpu, p, M, b, heads, schedule):

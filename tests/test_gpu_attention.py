@@ -201,3 +201,43 @@ def test_order_errors_leave_gpu_state_intact():
         pat.check()
     finally:
         pat.close()
+
+
+@pytest.mark.parametrize("d", [64, 72, 128])
+def test_distrifusion_schedule(d):
+    # patches in a random order each step; every other patch is seen at the previous step
+    wl = synth.AttnWorkload("distri", batch=1, heads=3, head_dim=d, grid_h=16, grid_w=40,
+                            n_patches=5, n_txt=20, n_layers=2, n_steps=3, ar_a=0.95, ar_b=0.3)
+    chk = run_workload(wl, full_check=lambda s, l, p: True, schedule=pa.PF_SCHED_DISTRIFUSION)
+    assert chk.n == 3 * 2 * 5
+
+
+def test_pipefusion_closer_to_fresh_than_distrifusion_on_gpu():
+    """Quality claim of the pages, measured on the GPU outputs of both schedules."""
+    wl = synth.AttnWorkload("claim", 1, 4, 64, 32, 32, 4, 16, 1, 3, 0.95, 0.3)
+    P = wl.patch_len
+    errs = {}
+    for sched in (pa.PF_SCHED_PIPEFUSION, pa.PF_SCHED_DISTRIFUSION):
+        gen = synth.AttnInputs(wl, seed=3, device="cuda")
+        pat = pa.PatchAttention(1, 4, 64, wl.n_img, 4, 16, 1, schedule=sched)
+        e = 0.0
+        try:
+            for s in range(3):
+                cur = gen.step_tensors(0)
+                if s == 0:
+                    pat.init_layer(0, cur["k"], cur["v"])
+                outs = []
+                for p in range(4):
+                    sl = slice(p * P, (p + 1) * P)
+                    outs.append(pat.step(0, p, cur["q"][:, sl].contiguous(), cur["k"][:, sl].contiguous(),
+                                         cur["v"][:, sl].contiguous(), cur["k_txt"], cur["v_txt"]))
+                if s == 2:
+                    o = f64(torch.cat(outs, dim=1)[0])
+                    fresh = oracle.attend(f64(cur["q"][0]), np.concatenate([f64(cur["k"][0]), f64(cur["k_txt"][0])]),
+                                          np.concatenate([f64(cur["v"][0]), f64(cur["v_txt"][0])]), wl.softmax_scale)
+                    e = float(np.sum((o - fresh) ** 2))
+            pat.check()
+        finally:
+            pat.close()
+        errs[sched] = e
+    assert errs[pa.PF_SCHED_PIPEFUSION] < errs[pa.PF_SCHED_DISTRIFUSION], errs

@@ -303,3 +303,74 @@ def test_key_order_does_not_matter():
     perm = rng.permutation(30)
     np.testing.assert_allclose(oracle.attend(q, k, v, 0.4), oracle.attend(q, k[perm], v[perm], 0.4),
                                rtol=1e-13, atol=1e-14)
+
+
+# ---------------------------------------------------------------- DistriFusion schedule
+
+
+def _df_args(steps, s):
+    cur, prev = steps[s], steps[s - 1]
+    return [f64(cur["q"]), f64(cur["k"]), f64(cur["v"]), f64(prev["k"]), f64(prev["v"]),
+            f64(cur["k_txt"]), f64(cur["v_txt"])]
+
+
+def test_distrifusion_single_patch_and_stale_equal_fresh_are_full_attention():
+    wl = _small_wl(n_patches=1)
+    steps = _gen_steps(wl, 2)
+    args = _df_args(steps, 1)
+    full = oracle.attend(args[0], np.concatenate([args[1], args[5]]), np.concatenate([args[2], args[6]]),
+                         wl.softmax_scale)
+    np.testing.assert_array_equal(oracle.distrifusion_attention(*args, 0, 1, wl.softmax_scale), full)
+    wl = _small_wl()
+    steps = _gen_steps(wl, 2, a=1.0, b=0.0)
+    args = _df_args(steps, 1)
+    full = oracle.attend(args[0], np.concatenate([args[1], args[5]]), np.concatenate([args[2], args[6]]),
+                         wl.softmax_scale)
+    for p in range(wl.n_patches):
+        np.testing.assert_array_equal(oracle.distrifusion_attention(*args, p, wl.n_patches, wl.softmax_scale),
+                                      full[p * wl.patch_len:(p + 1) * wl.patch_len])
+
+
+def test_distrifusion_sees_only_its_own_fresh_rows():
+    wl = _small_wl(n_patches=4, grid_h=4, grid_w=4)
+    args = _df_args(_gen_steps(wl, 2), 1)
+    plen = wl.patch_len
+    for p in range(wl.n_patches):
+        base = oracle.distrifusion_attention(*args, p, wl.n_patches, wl.softmax_scale)
+        for r in range(wl.n_patches):
+            rows = slice(r * plen, (r + 1) * plen)
+            a2 = [x.copy() for x in args]
+            a2[1][rows] += 1.0
+            a2[2][rows] += 1.0
+            fresh_changed = not np.array_equal(base, oracle.distrifusion_attention(*a2, p, wl.n_patches, wl.softmax_scale))
+            a3 = [x.copy() for x in args]
+            a3[3][rows] += 1.0
+            a3[4][rows] += 1.0
+            stale_changed = not np.array_equal(base, oracle.distrifusion_attention(*a3, p, wl.n_patches, wl.softmax_scale))
+            assert fresh_changed == (r == p) and stale_changed == (r != p), (p, r)
+
+
+def test_distrifusion_matches_pipefusion_on_last_patch_only_at_first_patch():
+    # patch 0: both schedules see stale rows for every other patch -> identical
+    wl = _small_wl()
+    args = _df_args(_gen_steps(wl, 2), 1)
+    np.testing.assert_array_equal(oracle.distrifusion_attention(*args, 0, wl.n_patches, wl.softmax_scale),
+                                  oracle.patch_attention(*args, 0, wl.n_patches, wl.softmax_scale))
+
+
+def test_pipefusion_stays_closer_to_fresh_attention_than_distrifusion():
+    """The pages' quality claim ("기술 요약: PipeFusion", 주요 기여 / 품질 보존: PipeFusion uses
+    fresh activations over a wider area than DistriFusion), on AR(1) synthetic activations:
+    the error against all-fresh attention, over a whole step, is smaller for PipeFusion."""
+    wl = _small_wl(n_patches=4, grid_h=8, grid_w=8, n_txt=4, heads=2, head_dim=16)
+    steps = _gen_steps(wl, 3)
+    for s in (1, 2):
+        args = _df_args(steps, s)
+        fresh = oracle.attend(args[0], np.concatenate([args[1], args[5]]), np.concatenate([args[2], args[6]]),
+                              wl.softmax_scale)
+        e_pf = e_df = 0.0
+        for p in range(wl.n_patches):
+            sl = slice(p * wl.patch_len, (p + 1) * wl.patch_len)
+            e_pf += np.sum((oracle.patch_attention(*args, p, wl.n_patches, wl.softmax_scale) - fresh[sl]) ** 2)
+            e_df += np.sum((oracle.distrifusion_attention(*args, p, wl.n_patches, wl.softmax_scale) - fresh[sl]) ** 2)
+        assert e_pf < e_df, (s, e_pf, e_df)
