@@ -112,6 +112,28 @@ pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
                              const void* k_p, const void* v_p, const void* k_txt,
                              const void* v_txt, void* o_p, void* stream);
 
+/* Joint attention for the text tokens (MM-DiT, named in "기술 요약: PipeFusion", 중요성 및
+ * 주장): the step's text queries attend to the layer's K/V buffer as it stands plus the text
+ * keys/values, softmax(scale Q_txt [K_buf;K_txt]^T) [V_buf;V_txt].  Called after the last
+ * patch of a step, the buffer holds that step's K/V everywhere.  The buffer is only read
+ * and the patch counter is not moved.
+ *   q_txt, k_txt, v_txt, o_txt : [B, T, H, d] bf16 (o_txt must not alias an input)
+ * Errors: PF_ERR_SHAPE if the configuration has no text tokens; PF_ERR_STATE before
+ * pf_kvbuf_init(layer). */
+pf_status pf_text_attn_step(pf_ctx* ctx, int layer, const void* q_txt, const void* k_txt,
+                            const void* v_txt, void* o_txt, void* stream);
+
+/* Per-head RMS normalisation of queries or keys, in place (the QK-norm of Flux-style DiTs):
+ * each head_dim vector x becomes x / sqrt(mean(x^2) + eps) * gain, computed in fp32 and
+ * rounded to bf16.
+ *   x         : device bf16, n_vectors contiguous vectors of head_dim elements
+ *               (e.g. [B, tokens, H, d] with n_vectors = B * tokens * H), 16-byte aligned
+ *   gain      : device bf16 [head_dim], or NULL for a gain of 1
+ *   eps       : > 0
+ * head_dim must be a multiple of 8 and at most 256. */
+pf_status pf_qk_rmsnorm(void* x, int64_t n_vectors, int head_dim, const void* gain, float eps,
+                        void* stream);
+
 /* Bytes of the optional attention workspace for this configuration (0 if cfg is invalid).
  * With a workspace set, a call may split each query tile's key range over several CTAs so
  * that the grid fills the GPU's SMs in near-whole waves; the parts are merged exactly in

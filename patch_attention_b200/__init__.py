@@ -37,7 +37,7 @@ EXPORTED = [
     "pf_get_state", "pf_set_state", "pf_workspace_bytes", "pf_set_workspace",
     "pf_cfg_workspace_bytes", "pf_cfg_combine_relmae", "pf_cfg_combine_relmae_static",
     "pf_check_device_status", "pf_status_string", "pf_version", "pf_switch_init",
-    "pf_switch_update",
+    "pf_switch_update", "pf_text_attn_step", "pf_qk_rmsnorm",
 ]
 
 PF_PHASE_WARMUP = 0
@@ -95,6 +95,8 @@ def _lib():
             "pf_cfg_combine_relmae_static": (i, [vp, vp, i, i64, f, vp, vp, vp, vp]),
             "pf_check_device_status": (i, [vp, vp]),
             "pf_status_string": (ctypes.c_char_p, [i]),
+            "pf_text_attn_step": (i, [vp, i, vp, vp, vp, vp, vp]),
+            "pf_qk_rmsnorm": (i, [vp, i64, i, vp, f, vp]),
             "pf_switch_init": (i, [ctypes.POINTER(pf_switch), f, i, f, i]),
             "pf_switch_update": (i, [ctypes.POINTER(pf_switch), f, ctypes.POINTER(i)]),
             "pf_version": (i, []),
@@ -185,6 +187,24 @@ def pf_patch_attn_step(ctx, layer: int, patch: int, q_p, k_p, v_p, k_txt, v_txt,
             _ptr(v_txt, bf, txt_shape, "v_txt"), _ptr(o_p, bf, patch_shape, "o_p"))
     _check(_lib().pf_patch_attn_step(ctx, layer, patch, *args, _stream(stream)),
            "pf_patch_attn_step")
+
+
+def pf_text_attn_step(ctx, layer: int, q_txt, k_txt, v_txt, o_txt, stream=None,
+                      txt_shape=None) -> None:
+    bf = torch.bfloat16
+    args = (_ptr(q_txt, bf, txt_shape, "q_txt"), _ptr(k_txt, bf, txt_shape, "k_txt"),
+            _ptr(v_txt, bf, txt_shape, "v_txt"), _ptr(o_txt, bf, txt_shape, "o_txt"))
+    _check(_lib().pf_text_attn_step(ctx, layer, *args, _stream(stream)), "pf_text_attn_step")
+
+
+def pf_qk_rmsnorm(x: torch.Tensor, gain: Optional[torch.Tensor] = None, eps: float = 1e-6,
+                  stream=None) -> None:
+    """Normalise every head vector (last dimension) of the bf16 tensor x in place."""
+    d = x.shape[-1]
+    xp = _ptr(x, torch.bfloat16, None, "x")
+    gp = _ptr(gain, torch.bfloat16, (d,), "gain")
+    _check(_lib().pf_qk_rmsnorm(xp, x.numel() // d, d, gp, float(eps), _stream(stream)),
+           "pf_qk_rmsnorm")
 
 
 def pf_workspace_bytes(cfg: pf_config) -> int:
@@ -314,6 +334,13 @@ class PatchAttention:
             k_txt = v_txt = None
         pf_patch_attn_step(self.ctx, layer, patch, q_p, k_p, v_p, k_txt, v_txt, out, stream,
                            self.patch_shape, self.txt_shape)
+        return out
+
+    def text_step(self, layer, q_txt, k_txt, v_txt, out=None, stream=None):
+        """Text-token queries against the layer buffer as it stands plus the text tokens."""
+        if out is None:
+            out = torch.empty(self.txt_shape, dtype=torch.bfloat16, device=q_txt.device)
+        pf_text_attn_step(self.ctx, layer, q_txt, k_txt, v_txt, out, stream, self.txt_shape)
         return out
 
     def buffer_kv(self, layer, half=0):

@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libpatchattn.so")
 OBJDIR = os.path.join(HERE, "_build")
 
-SOURCES = ["attn_fwd.cu", "cfg_combine.cu", "kvbuf_copy.cu", "pf_api.cpp"]
+SOURCES = ["attn_fwd.cu", "cfg_combine.cu", "kvbuf_copy.cu", "qk_rmsnorm.cu", "pf_api.cpp"]
 HEADERS = ["pf_internal.h", "sm100_ptx.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

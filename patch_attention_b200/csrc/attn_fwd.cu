@@ -106,10 +106,10 @@ struct Segments {
   int plen, lo_len, hi_row0, hi_len, txt_len;
 
   __device__ void init(const AttnParams& p) {
-    plen = p.plen;
-    lo_len = p.patch * p.plen;
-    hi_row0 = (p.patch + 1) * p.plen;
-    hi_len = p.n_img - hi_row0;
+    plen = p.fresh_rows;
+    lo_len = p.lo_len;
+    hi_row0 = p.hi_row0;
+    hi_len = p.hi_len;
     txt_len = p.n_txt;
     n_fresh = (plen + kRows - 1) / kRows;
     n_lo = (lo_len + kRows - 1) / kRows;
@@ -332,8 +332,10 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
   }
   if (warp == kWarpLoad && lane == 0) {
     prefetch_tmap(&p.tm_q);
-    prefetch_tmap(&p.tm_kf);
-    prefetch_tmap(&p.tm_vf);
+    if (p.fresh_rows > 0) {
+      prefetch_tmap(&p.tm_kf);
+      prefetch_tmap(&p.tm_vf);
+    }
     prefetch_tmap(&p.tm_kb);
     prefetch_tmap(&p.tm_vb);
     if (p.n_txt > 0) {
@@ -717,8 +719,8 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
         tc_fence_after();
         const int rloc = wq * 32 + lane;
         const int row = q0 + t * kRows + rloc;
-        uint16_t* dst = p.o + ((static_cast<size_t>(b) * p.plen + row) * p.heads + h) * D;
-        const bool in_range = row < p.plen;
+        uint16_t* dst = p.o + ((static_cast<size_t>(b) * p.q_rows + row) * p.heads + h) * D;
+        const bool in_range = row < p.q_rows;
         if (p.n_split == 1) {
           const float inv = 1.f / l;
 #pragma unroll
@@ -834,10 +836,9 @@ __global__ void zero_u32_kernel(unsigned* p, size_t n) {
 
 int attn_tiles_per_cta(int plen) { return plen > kRows ? 2 : 1; }
 
-int attn_context_tiles(int plen, int n_img, int n_txt, int patch) {
+int attn_context_tiles(int fresh_rows, int lo_len, int hi_len, int n_txt) {
   auto tiles = [](long long n) { return static_cast<int>((n + kRows - 1) / kRows); };
-  return tiles(plen) + tiles(static_cast<long long>(patch) * plen) +
-         tiles(n_img - static_cast<long long>(patch + 1) * plen) + tiles(n_txt);
+  return tiles(fresh_rows) + tiles(lo_len) + tiles(hi_len) + tiles(n_txt);
 }
 
 int attn_choose_split(int n_pairs, int n_tiles, int n_sms, int max_split) {
@@ -875,7 +876,7 @@ cudaError_t launch_zero_u32(unsigned* p, size_t n, cudaStream_t stream) {
 }
 
 cudaError_t launch_patch_attn(const AttnParams& p, cudaStream_t stream) {
-  const bool two = p.plen > kRows;
+  const bool two = p.q_rows > kRows;
   switch (p.head_dim) {
     case 64: return two ? launch_one<64, 2>(p, stream) : launch_one<64, 1>(p, stream);
     case 72: return two ? launch_one<72, 2>(p, stream) : launch_one<72, 1>(p, stream);

@@ -97,33 +97,81 @@ bool make_map(CUtensorMap* m, const void* base, int batch, int rows, int heads, 
 
 pf_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PF_OK : PF_ERR_CUDA; }
 
-int pairs_of(const pf_config& c) {
-  const int plen = c.n_img / c.n_patches;
-  const int nq = pf::attn_tiles_per_cta(plen);
-  const int groups = (plen + nq * 128 - 1) / (nq * 128);
+// (batch, head, query-tile group) pairs of a call with q_rows query rows
+int pairs_for(const pf_config& c, int q_rows) {
+  const int nq = pf::attn_tiles_per_cta(q_rows);
+  const int groups = (q_rows + nq * 128 - 1) / (nq * 128);
   return c.batch * c.heads * groups;
+}
+
+int pairs_of(const pf_config& c) {
+  const int a = pairs_for(c, c.n_img / c.n_patches);
+  const int b = c.n_txt > 0 ? pairs_for(c, c.n_txt) : 0;
+  return a > b ? a : b;
 }
 
 constexpr int kAssumedSms = 148;
 
-// Counters first (fixed place), then the partial slots.
+// Counters first (fixed place, sized for the larger of patch and text-query calls), then the
+// partial slots.
 size_t counter_bytes(int pairs) { return ((static_cast<size_t>(pairs) * 2 * 4 + 255) / 256) * 256; }
 
 size_t workspace_for(const pf_config& c, int n_sms) {
   const int plen = c.n_img / c.n_patches;
-  const int pairs = pairs_of(c);
+  const size_t cb = counter_bytes(pairs_of(c));
   size_t best = 0;
-  for (int p = 0; p < c.n_patches; ++p) {
-    const int tiles = pf::attn_context_tiles(plen, c.n_img, c.n_txt, p);
+  auto consider = [&](int q_rows, int tiles) {
+    const int pairs = pairs_for(c, q_rows);
     const int k = pf::attn_choose_split(pairs, tiles, n_sms, 1 << 30);
-    const size_t b = k > 1 ? counter_bytes(pairs) + pf::attn_workspace_bytes(pairs, c.head_dim, k) : 0;
+    const size_t b = k > 1 ? cb + pf::attn_workspace_bytes(pairs, c.head_dim, k) : 0;
     if (b > best) best = b;
+  };
+  for (int p = 0; p < c.n_patches; ++p) {
+    consider(plen, pf::attn_context_tiles(plen, p * plen, c.n_img - (p + 1) * plen, c.n_txt));
     if (plen % 128 == 0) break;  // every patch has the same tile count
   }
+  if (c.n_txt > 0) consider(c.n_txt, pf::attn_context_tiles(0, c.n_img, 0, c.n_txt));
   return best;
 }
 
 bool layer_ok(const pf_ctx* ctx, int layer) { return layer >= 0 && layer < ctx->cfg.n_layers; }
+
+// Fill the fields common to every attention call (sizes, scale, work decomposition and
+// key-range split) and launch.  p carries the tensor maps, pointers and segments.
+cudaError_t launch_attention(pf_ctx* ctx, pf::AttnParams& p, void* stream) {
+  const pf_config& c = ctx->cfg;
+  p.batch = c.batch;
+  p.heads = c.heads;
+  p.n_img = c.n_img;
+  p.n_txt = c.n_txt;
+  p.head_dim = c.head_dim;
+  p.scale_log2 = ctx->scale * 1.4426950408889634f;
+  const int nq = pf::attn_tiles_per_cta(p.q_rows);
+  p.n_groups = (p.q_rows + nq * 128 - 1) / (nq * 128);
+  p.n_pairs = c.batch * c.heads * p.n_groups;
+  p.n_split = 1;
+  if (ctx->ws != nullptr) {
+    if (ctx->n_sms == 0) {
+      int dev = 0, n = 0;
+      if (cudaGetDevice(&dev) == cudaSuccess &&
+          cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+        ctx->n_sms = n;
+      else
+        ctx->n_sms = kAssumedSms;
+    }
+    const int tiles = pf::attn_context_tiles(p.fresh_rows, p.lo_len, p.hi_len, c.n_txt);
+    const size_t cb = counter_bytes(pairs_of(c));
+    int cap = 1;  // most parts the workspace can hold
+    while (cap < 16 && cb + pf::attn_workspace_bytes(p.n_pairs, c.head_dim, cap + 1) <= ctx->ws_bytes)
+      ++cap;
+    p.n_split = pf::attn_choose_split(p.n_pairs, tiles, ctx->n_sms, cap);
+    if (p.n_split > 1) {
+      p.ws_cnt = reinterpret_cast<unsigned*>(ctx->ws);
+      p.ws_part = reinterpret_cast<float*>(ctx->ws + cb);
+    }
+  }
+  return pf::launch_patch_attn(p, static_cast<cudaStream_t>(stream));
+}
 
 // K/V regions of a layer's buffer: half 0 is [K | V]; DistriFusion adds half 1 [K | V].
 uint8_t* region(const pf_ctx* ctx, int layer, int half, int kv) {
@@ -230,40 +278,14 @@ pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
   p.k_dst = reinterpret_cast<uint16_t*>(region(ctx, layer, write, 0));
   p.v_dst = reinterpret_cast<uint16_t*>(region(ctx, layer, write, 1));
   p.o = static_cast<uint16_t*>(o_p);
-  p.batch = c.batch;
-  p.heads = c.heads;
   p.plen = plen;
-  p.n_img = c.n_img;
-  p.n_txt = c.n_txt;
   p.patch = patch;
-  p.head_dim = d;
-  p.scale_log2 = ctx->scale * 1.4426950408889634f;
-  const int nq = pf::attn_tiles_per_cta(plen);
-  p.n_groups = (plen + nq * 128 - 1) / (nq * 128);
-  p.n_pairs = c.batch * c.heads * p.n_groups;
-  p.n_split = 1;
-  if (ctx->ws != nullptr) {
-    if (ctx->n_sms == 0) {
-      int dev = 0, n = 0;
-      if (cudaGetDevice(&dev) == cudaSuccess &&
-          cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
-        ctx->n_sms = n;
-      else
-        ctx->n_sms = kAssumedSms;
-    }
-    const int tiles = pf::attn_context_tiles(plen, c.n_img, c.n_txt, patch);
-    const size_t cb = counter_bytes(p.n_pairs);
-    int cap = 1;  // most parts the workspace can hold
-    while (cap < 16 && cb + pf::attn_workspace_bytes(p.n_pairs, d, cap + 1) <= ctx->ws_bytes) ++cap;
-    p.n_split = pf::attn_choose_split(p.n_pairs, tiles, ctx->n_sms, cap);
-    if (p.n_split > 1) {
-      p.ws_cnt = reinterpret_cast<unsigned*>(ctx->ws);
-      p.ws_part = reinterpret_cast<float*>(ctx->ws + cb);
-    }
-  }
-
-  cudaError_t e = pf::launch_patch_attn(p, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return PF_ERR_CUDA;
+  p.q_rows = plen;
+  p.fresh_rows = plen;
+  p.lo_len = patch * plen;
+  p.hi_row0 = (patch + 1) * plen;
+  p.hi_len = c.n_img - (patch + 1) * plen;
+  if (launch_attention(ctx, p, stream) != cudaSuccess) return PF_ERR_CUDA;
 
   if (pipefusion) {
     ctx->next_patch[layer] = (patch + 1) % c.n_patches;
@@ -279,6 +301,47 @@ pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
     ctx->next_patch[layer] = ctx->seen_count[layer];
   }
   return PF_OK;
+}
+
+pf_status pf_text_attn_step(pf_ctx* ctx, int layer, const void* q_txt, const void* k_txt,
+                            const void* v_txt, void* o_txt, void* stream) {
+  if (!ctx) return PF_ERR_INVALID_ARG;
+  const pf_config& c = ctx->cfg;
+  if (!layer_ok(ctx, layer)) return PF_ERR_INVALID_ARG;
+  if (c.n_txt == 0) return PF_ERR_SHAPE;
+  if (!q_txt || !k_txt || !v_txt || !o_txt) return PF_ERR_INVALID_ARG;
+  if (!aligned16(q_txt) || !aligned16(k_txt) || !aligned16(v_txt) || !aligned16(o_txt))
+    return PF_ERR_ALIGN;
+  if (!ctx->initialised[layer]) return PF_ERR_STATE;
+  const int d = c.head_dim;
+  const int read = ctx->read_half[layer];
+  pf::AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (!make_map(&p.tm_q, q_txt, c.batch, c.n_txt, c.heads, d) ||
+      !make_map(&p.tm_kb, region(ctx, layer, read, 0), c.batch, c.n_img, c.heads, d) ||
+      !make_map(&p.tm_vb, region(ctx, layer, read, 1), c.batch, c.n_img, c.heads, d) ||
+      !make_map(&p.tm_kt, k_txt, c.batch, c.n_txt, c.heads, d) ||
+      !make_map(&p.tm_vt, v_txt, c.batch, c.n_txt, c.heads, d))
+    return PF_ERR_CUDA;
+  p.o = static_cast<uint16_t*>(o_txt);
+  p.plen = c.n_img / c.n_patches;
+  p.q_rows = c.n_txt;   // text queries
+  p.fresh_rows = 0;     // no fresh patch rows, no scatter (k_dst stays null)
+  p.lo_len = c.n_img;   // the whole buffer as it stands
+  p.hi_row0 = c.n_img;
+  p.hi_len = 0;
+  if (launch_attention(ctx, p, stream) != cudaSuccess) return PF_ERR_CUDA;
+  return PF_OK;
+}
+
+pf_status pf_qk_rmsnorm(void* x, int64_t n_vectors, int head_dim, const void* gain, float eps,
+                        void* stream) {
+  if (!x || n_vectors < 0) return PF_ERR_INVALID_ARG;
+  if (head_dim < 8 || head_dim > 256 || head_dim % 8 != 0) return PF_ERR_SHAPE;
+  if (!(eps > 0.f) || !std::isfinite(eps)) return PF_ERR_INVALID_ARG;
+  if (!aligned16(x) || (gain && !aligned16(gain))) return PF_ERR_ALIGN;
+  return from_cuda(pf::launch_qk_rmsnorm(x, n_vectors, head_dim, gain, eps,
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 pf_status pf_get_state(const pf_ctx* ctx, int layer, int* next_patch) {

@@ -24,9 +24,15 @@ struct AttnParams {
   const uint16_t* v_p;
   uint16_t* k_dst;      // scatter destination: buffer rows of the patch (K region base)
   uint16_t* v_dst;      // (V region base); both null => no scatter
-  uint16_t* o;          // O_p [B, P, H, d]
+  uint16_t* o;          // O [B, q_rows, H, d]
   int batch, heads, plen, n_img, n_txt, patch, head_dim;
   float scale_log2;     // softmax scale * log2(e)
+  // Queries and context: q_rows query rows (tm_q); the context is the fresh rows
+  // [0, fresh_rows) of tm_kf/tm_vf, buffer rows [0, lo_len) and [hi_row0, hi_row0 + hi_len),
+  // then the n_txt text rows.  A patch micro-step has q_rows = fresh_rows = plen and the
+  // buffer minus the patch's own rows; a text-query call has q_rows = n_txt, no fresh rows
+  // and the whole buffer.
+  int q_rows, fresh_rows, lo_len, hi_row0, hi_len;
   // Work decomposition: a "pair" is one (batch, head, group of NQ query tiles); its key
   // range is split into n_split contiguous parts, one CTA per (pair, part).
   int n_groups;         // query-tile groups per (batch, head)
@@ -38,8 +44,8 @@ struct AttnParams {
 
 // Query tiles per CTA chosen for a patch length (1 or 2).
 int attn_tiles_per_cta(int plen);
-// Number of 128-row context tiles of one micro-step.
-int attn_context_tiles(int plen, int n_img, int n_txt, int patch);
+// Number of 128-row context tiles of a call with the given segment lengths.
+int attn_context_tiles(int fresh_rows, int lo_len, int hi_len, int n_txt);
 // Key-range parts per (batch, head, query-tile group) for a call, given the number of SMs
 // and the number of parts the workspace can hold.
 int attn_choose_split(int n_pairs, int n_tiles, int n_sms, int max_split);
@@ -50,6 +56,10 @@ cudaError_t launch_zero_u32(unsigned* p, size_t n, cudaStream_t stream);
 
 // Launch the fused scatter + attention kernel.  Returns the launch error.
 cudaError_t launch_patch_attn(const AttnParams& p, cudaStream_t stream);
+
+// In-place per-head RMS normalisation of bf16 vectors (head_dim multiple of 8, <= 256).
+cudaError_t launch_qk_rmsnorm(void* x, long long n_vectors, int head_dim, const void* gain,
+                              float eps, cudaStream_t stream);
 
 // Start-up copy of full-spatial K/V into a layer buffer (16-byte vectors).
 cudaError_t launch_kvbuf_copy(const void* k_src, const void* v_src, void* k_dst, void* v_dst,
