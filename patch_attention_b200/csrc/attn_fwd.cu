@@ -133,11 +133,6 @@ struct Segments {
     j -= n_hi;
     src = 2; row0 = j * kRows; nvalid = min(kRows, txt_len - row0);
   }
-  __device__ int nvalid(int j) const {
-    int s, r, n;
-    tile(j, s, r, n);
-    return n;
-  }
 };
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -203,15 +198,21 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
-// Maximum of 128 values: 8 independent chains, then a tree.
+// Maximum of 128 values: 8 independent chains of three-input maxima, then a tree.
 __device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) {
   float mv[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) mv[k] = __uint_as_float(s[k]);
 #pragma unroll
-  for (int k = 8; k < 128; ++k) mv[k & 7] = fmaxf(mv[k & 7], __uint_as_float(s[k]));
-  return fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
-               fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
+  for (int k = 8; k < 120; k += 2)
+    mv[(k >> 1) & 7] = max3(mv[(k >> 1) & 7], __uint_as_float(s[k]), __uint_as_float(s[k + 1]));
+  mv[0] = max3(mv[0], mv[4], __uint_as_float(s[120]));
+  mv[1] = max3(mv[1], mv[5], __uint_as_float(s[121]));
+  mv[2] = max3(mv[2], mv[6], __uint_as_float(s[122]));
+  mv[3] = max3(mv[3], mv[7], __uint_as_float(s[123]));
+  mv[0] = max3(mv[0], __uint_as_float(s[124]), __uint_as_float(s[125]));
+  mv[1] = max3(mv[1], __uint_as_float(s[126]), __uint_as_float(s[127]));
+  return max3(mv[0], mv[1], fmaxf(mv[2], mv[3]));
 }
 
 // p_k = 2^(s_k c - m), packed to bf16 pairs; returns the fp32 sum.  POLY of every 8 pairs
@@ -235,6 +236,20 @@ __device__ __forceinline__ void exact_exps(const uint32_t (&s)[128], float c, fl
   lsum = a.x + a.y;
 }
 
+// exact_exps over the column pairs [K0, K1) only, accumulating the fp32 sums into acc (the
+// caller adds acc up): lets a caller place other work between two halves of a row.
+template <int POLY, int K0, int K1>
+__device__ __forceinline__ void exps_span(const uint32_t (&s)[128], float2 cc, float2 nm,
+                                          uint32_t (&pk)[64], float2 (&acc)[4]) {
+#pragma unroll
+  for (int k = K0; k < K1; ++k) {
+    const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), cc, nm);
+    const float2 p = (k & 7) < POLY ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
+    acc[k & 3] = __fadd2_rn(acc[k & 3], p);
+    pk[k] = pack_bf16(p.x, p.y);
+  }
+}
+
 // Same as exact_exps against the current reference m, with POLY of every 8 pairs of
 // columns exponentiated on the FMA pipe; returns max_k (s_k c - m) so the caller can
 // check that no p_k exceeded 2^8.
@@ -248,7 +263,7 @@ __device__ __forceinline__ float speculative_exps(const uint32_t (&s)[128], floa
 #pragma unroll
   for (int k = 0; k < 64; ++k) {
     const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), cc, nm);
-    xm[k & 3] = fmaxf(xm[k & 3], fmaxf(x.x, x.y));
+    xm[k & 3] = max3(xm[k & 3], x.x, x.y);
     float2 p;
     if ((k & 7) < POLY) {
       p = exp2_poly2(x);
@@ -458,11 +473,13 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
             const int iK = 2 * (j + 1), sK = iK % S;
             if (!(ok = mbar_wait(smem_u32(kv_full + sK), (iK / S) & 1, abort, kWaitNs))) break;
             tc_fence_after();
+            PF_TRACE_AT(4, 0, j + 1);
             for (int t = 0; t < NQ; ++t) {
               if (!(ok = mbar_wait(smem_u32(s_free + t), j & 1, abort, kWaitNs))) break;
               tc_fence_after();
               issue_qk(t, sK);
               mma_commit(smem_u32(s_full + t));
+              PF_TRACE_AT(3, t, j + 1);
             }
             if (!ok) break;
             mma_commit(smem_u32(kv_empty + sK));
@@ -470,9 +487,11 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
           const int iV = 2 * j + 1, sV = iV % S;
           if (!(ok = mbar_wait(smem_u32(kv_full + sV), (iV / S) & 1, abort, kWaitNs))) break;
           tc_fence_after();
+          PF_TRACE_AT(9, 0, j);
           for (int t = 0; t < NQ; ++t) {
             if (!(ok = mbar_wait(smem_u32(p_full + t), j & 1, abort, kWaitNs))) break;
             tc_fence_after();
+            PF_TRACE_AT(2, t, j);
             issue_pv(t, sV, j > 0);
             mma_commit(smem_u32(pv_done + t));
           }
@@ -577,6 +596,21 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
     float m = -INFINITY;  // reference row maximum, already scaled to log2 units
     float l = 0.f;
     bool ok = true;
+    // Local indices of this CTA's context tiles with fewer than 128 valid rows (the last tile
+    // of a segment whose length is not a multiple of 128; -1 if not in range) and their
+    // valid row counts, so the loop needs no segment arithmetic.
+    int rag_j[4], rag_nv[4];
+    {
+      const int ends[4] = {seg.n_fresh, seg.n_fresh + seg.n_lo, seg.n_fresh + seg.n_lo + seg.n_hi,
+                           seg.total()};
+      const int lens[4] = {seg.plen, seg.lo_len, seg.hi_len, seg.txt_len};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int e = ends[k] - 1;
+        rag_nv[k] = lens[k] % kRows;
+        rag_j[k] = (rag_nv[k] != 0 && e >= j0 && e < j1) ? e - j0 : -1;
+      }
+    }
     for (int j = 0; j < n_tiles; ++j) {
       ok = mbar_wait(smem_u32(s_full + t), j & 1, abort, kWaitNs);
       ok = __all_sync(0xffffffffu, ok);
@@ -591,7 +625,10 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
       tmem_wait_ld();
       reg_fence<128>(s);
       if (wq == 0 && lane == 0) PF_TRACE_AT(5, t, j);
-      const int nv = seg.nvalid(j0 + j);
+      int nv = kRows;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (j == rag_j[k]) nv = rag_nv[k];
       uint32_t pk[64];
       float lsum;
       if constexpr (kSepP) {
@@ -605,6 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
             if (k >= nv) s[k] = __float_as_uint(-INFINITY);
         }
         const float mxs = row_max128(s) * c;
+        if (wq == 0 && lane == 0) PF_TRACE_AT(6, t, j);
         bool pv_seen = (j == 0);  // PV of the previous tile done: O stable, P columns free
         if (mxs > m + 8.f) {
           const float alpha = ex2(m - mxs);
@@ -628,17 +666,27 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
           }
           m = mxs;
         }
-        if (nv < kRows)
-          exact_exps<0>(s, c, m, pk, lsum);
-        else
-          exact_exps<kPolyPairs<D>>(s, c, m, pk, lsum);
+        // Masked keys (-inf) give exactly 0 on the special-function unit and 2^-125 on the
+        // polynomial, which is below any sum that includes the row maximum's own term (1),
+        // so ragged tiles use the same mix.  Half way through, probe (without blocking)
+        // whether PV of the previous tile has released the P columns.
+        {
+          const float2 cc = make_float2(c, c), nm = make_float2(-m, -m);
+          float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                           make_float2(0.f, 0.f)};
+          exps_span<kPolyPairs<D>, 0, 32>(s, cc, nm, pk, acc);
+          if (!pv_seen) pv_seen = mbar_test_wait_all(smem_u32(pv_done + t), (j - 1) & 1);
+          exps_span<kPolyPairs<D>, 32, 64>(s, cc, nm, pk, acc);
+          const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+          lsum = a.x + a.y;
+        }
         l += lsum;
         if (!pv_seen) {
           ok = mbar_wait(smem_u32(pv_done + t), (j - 1) & 1, abort, kWaitNs);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
-          tc_fence_after();
         }
+        tc_fence_after();
         if (wq == 0 && lane == 0) PF_TRACE_AT(7, t, j);
         tmem_st32(tO + 64, pk);
         tmem_st32(tO + 96, pk + 32);

@@ -72,6 +72,21 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t par
   return ok != 0;
 }
 
+// Non-blocking: whether the phase of `bar` with the given parity has completed, as seen by
+// every lane of the warp (one vote, so the answer is warp-uniform).
+__device__ __forceinline__ bool mbar_test_wait_all(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "vote.sync.all.pred q, p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase of `bar` with the given parity has completed.  Bounded: after
 // `limit_ns`, or once *abort becomes non-zero (abort may be null), give up and return
 // false.  Between checks the thread is suspended in hardware, for at most 0.5 ms each.
@@ -263,6 +278,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, int b_mn_maj
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Maximum of three floats in one instruction (three-input max.f32, sm_100 and later).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float y;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
   return y;
 }
 
