@@ -53,6 +53,18 @@ __device__ unsigned int g_watchdog = 0;
 constexpr int kTraceTiles = 512;
 // 9 MMA issuer sees the V tile of j-1, 10 producer issued the K (t=0) / V (t=1) tile j.
 __device__ unsigned long long g_trace[11 * 2 * kTraceTiles];
+// Per CTA of the latest launch: SM id, start and end (global timer, ns).
+constexpr int kTraceCtas = 4096;
+__device__ unsigned long long g_cta[3 * kTraceCtas];
+#define PF_TRACE_CTA(slot)                                                                 \
+  do {                                                                                     \
+    if (threadIdx.x == 0 && blockIdx.x < kTraceCtas) {                                     \
+      unsigned smid;                                                                       \
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));                                    \
+      g_cta[3 * blockIdx.x] = smid;                                                        \
+      g_cta[3 * blockIdx.x + (slot)] = globaltimer_ns();                                   \
+    }                                                                                      \
+  } while (0)
 #define PF_TRACE_AT(ev, t, j)                                                              \
   do {                                                                                     \
     if (blockIdx.x == 0 && (j) < kTraceTiles) g_trace[((ev) * 2 + (t)) * kTraceTiles + (j)] = clock64(); \
@@ -60,6 +72,9 @@ __device__ unsigned long long g_trace[11 * 2 * kTraceTiles];
 #else
 #define PF_TRACE_AT(ev, t, j) \
   do {                        \
+  } while (0)
+#define PF_TRACE_CTA(slot) \
+  do {                     \
   } while (0)
 #endif
 
@@ -315,6 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  PF_TRACE_CTA(1);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int part = blockIdx.x / p.n_pairs;
@@ -809,37 +825,49 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
           }
           named_bar_sync(1 + t, kRows);
           if (s_last[t]) {
-            // merge every part of this query tile
-            float wgt[kMaxSplit];
-            float mref = -INFINITY;
+            // Merge every part of this query tile.  The loads are arranged so that each
+            // round trip to L2 fetches a whole 64-column block of one part's row (or every
+            // part's m and l), instead of one dependent round per 8 columns and part.
+            float mref = -INFINITY, lsum = 0.f;
+#pragma unroll 4
             for (int i = 0; i < p.n_split; ++i)
               mref = fmaxf(mref, __ldcg(slot0 + i * slot_elems + D * kRows + rloc));
-            float lsum = 0.f;
-            for (int i = 0; i < kMaxSplit; ++i) {
-              if (i < p.n_split) {
-                const float* si = slot0 + i * slot_elems;
-                wgt[i] = ex2(__ldcg(si + D * kRows + rloc) - mref);
-                lsum += wgt[i] * __ldcg(si + (D + 1) * kRows + rloc);
-              } else {
-                wgt[i] = 0.f;
-              }
+#pragma unroll 4
+            for (int i = 0; i < p.n_split; ++i) {
+              const float* si = slot0 + i * slot_elems;
+              lsum += ex2(__ldcg(si + D * kRows + rloc) - mref) * __ldcg(si + (D + 1) * kRows + rloc);
             }
             const float inv = 1.f / lsum;
-#pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 8) {
-              float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-              for (int i = 0; i < p.n_split; ++i) {
-                const float* si = slot0 + i * slot_elems + c0 * kRows + rloc;
 #pragma unroll
-                for (int k = 0; k < 8; ++k) acc[k] += wgt[i] * __ldcg(si + k * kRows);
+            for (int cb = 0; cb < D; cb += 64) {
+              constexpr int kBlock = 64;
+              const int nc = D - cb < kBlock ? D - cb : kBlock;  // constant once unrolled
+              float acc[kBlock];
+#pragma unroll
+              for (int k = 0; k < kBlock; ++k) acc[k] = 0.f;
+              for (int i = 0; i < p.n_split; ++i) {
+                const float* si = slot0 + i * slot_elems + rloc;
+                float v[kBlock];
+#pragma unroll
+                for (int k = 0; k < kBlock; ++k)
+                  if (k < nc) v[k] = __ldcg(si + (cb + k) * kRows);
+                const float w = ex2(__ldcg(si + D * kRows) - mref) * inv;
+#pragma unroll
+                for (int k = 0; k < kBlock; ++k)
+                  if (k < nc) acc[k] = fmaf(w, v[k], acc[k]);
               }
               if (in_range) {
-                uint4 w0;
-                w0.x = pack_bf16(acc[0] * inv, acc[1] * inv);
-                w0.y = pack_bf16(acc[2] * inv, acc[3] * inv);
-                w0.z = pack_bf16(acc[4] * inv, acc[5] * inv);
-                w0.w = pack_bf16(acc[6] * inv, acc[7] * inv);
-                *reinterpret_cast<uint4*>(dst + c0) = w0;
+#pragma unroll
+                for (int k = 0; k < kBlock; k += 8) {
+                  if (k < nc) {
+                    uint4 w0;
+                    w0.x = pack_bf16(acc[k + 0], acc[k + 1]);
+                    w0.y = pack_bf16(acc[k + 2], acc[k + 3]);
+                    w0.z = pack_bf16(acc[k + 4], acc[k + 5]);
+                    w0.w = pack_bf16(acc[k + 6], acc[k + 7]);
+                    *reinterpret_cast<uint4*>(dst + cb + k) = w0;
+                  }
+                }
               }
             }
           }
@@ -853,6 +881,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
 
   tc_fence_before();
   __syncthreads();
+  PF_TRACE_CTA(2);
   if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -937,6 +966,10 @@ cudaError_t launch_patch_attn(const AttnParams& p, cudaStream_t stream) {
 extern "C" int pf_trace_read(unsigned long long* dst, size_t n) {
   if (n > sizeof(g_trace) / sizeof(g_trace[0])) n = sizeof(g_trace) / sizeof(g_trace[0]);
   return static_cast<int>(cudaMemcpyFromSymbol(dst, g_trace, n * sizeof(unsigned long long)));
+}
+extern "C" int pf_trace_cta_read(unsigned long long* dst, size_t n) {
+  if (n > sizeof(g_cta) / sizeof(g_cta[0])) n = sizeof(g_cta) / sizeof(g_cta[0]);
+  return static_cast<int>(cudaMemcpyFromSymbol(dst, g_cta, n * sizeof(unsigned long long)));
 }
 #endif
 
