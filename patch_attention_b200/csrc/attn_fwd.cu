@@ -627,10 +627,13 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
         rag_j[k] = (rag_nv[k] != 0 && e >= j0 && e < j1) ? e - j0 : -1;
       }
     }
+    bool s_ready = false;  // separate-P layout: S(j) was seen complete at the end of tile j-1
     for (int j = 0; j < n_tiles; ++j) {
-      ok = mbar_wait(smem_u32(s_full + t), j & 1, abort, kWaitNs);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
+      if (!s_ready) {
+        ok = mbar_wait(smem_u32(s_full + t), j & 1, abort, kWaitNs);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+      }
       tc_fence_after();
       if (wq == 0 && lane == 0) PF_TRACE_AT(0, t, j);
       uint32_t s[128];
@@ -657,52 +660,57 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
           for (int k = 0; k < 128; ++k)
             if (k >= nv) s[k] = __float_as_uint(-INFINITY);
         }
+        // Reference maximum, updated without a branch (the O rescale it may need is done
+        // after the exponentials, before P is published).
         const float mxs = row_max128(s) * c;
         if (wq == 0 && lane == 0) PF_TRACE_AT(6, t, j);
-        bool pv_seen = (j == 0);  // PV of the previous tile done: O stable, P columns free
-        if (mxs > m + 8.f) {
-          const float alpha = ex2(m - mxs);
-          l *= alpha;
-          if (j > 0) {
-            ok = mbar_wait(smem_u32(pv_done + t), (j - 1) & 1, abort, kWaitNs);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            tc_fence_after();
-            pv_seen = true;
-#pragma unroll
-            for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
-              uint32_t o[16];
-              tmem_ld16(tO + c0, o);
-              tmem_wait_ld();
-              reg_fence<16>(o);
-#pragma unroll
-              for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-              tmem_st16(tO + c0, o);
-            }
-          }
-          m = mxs;
-        }
+        const bool grow = mxs > m + 8.f;
+        const float alpha = grow ? ex2(m - mxs) : 1.f;
+        l *= alpha;
+        m = grow ? mxs : m;
+        // P(j) may overwrite P(j-1) only once PV(j-1) has read it.  QK(j+1) was issued by
+        // the same thread after PV(j-1) and the tensor pipe completes in order, so S(j+1)
+        // being complete implies it -- and S(j+1) is what the next tile waits for anyway.
+        // The last tile waits for PV(j-1) itself.  The barrier is probed half way through
+        // the exponentials so that the wait is usually already over.
+        const bool has_next = j + 1 < n_tiles;
+        const uint32_t gate = has_next ? smem_u32(s_full + t) : smem_u32(pv_done + t);
+        const uint32_t gate_par = has_next ? static_cast<uint32_t>((j + 1) & 1)
+                                           : static_cast<uint32_t>((j - 1) & 1);
+        bool gate_ok = !has_next && j == 0;  // a single tile: nothing to wait for
         // Masked keys (-inf) give exactly 0 on the special-function unit and 2^-125 on the
         // polynomial, which is below any sum that includes the row maximum's own term (1),
-        // so ragged tiles use the same mix.  Half way through, probe (without blocking)
-        // whether PV of the previous tile has released the P columns.
+        // so ragged tiles use the same mix.
         {
           const float2 cc = make_float2(c, c), nm = make_float2(-m, -m);
           float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                            make_float2(0.f, 0.f)};
           exps_span<kPolyPairs<D>, 0, 32>(s, cc, nm, pk, acc);
-          if (!pv_seen) pv_seen = mbar_test_wait_all(smem_u32(pv_done + t), (j - 1) & 1);
+          if (!gate_ok) gate_ok = mbar_test_wait_all(gate, gate_par);
           exps_span<kPolyPairs<D>, 32, 64>(s, cc, nm, pk, acc);
           const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
           lsum = a.x + a.y;
         }
         l += lsum;
-        if (!pv_seen) {
-          ok = mbar_wait(smem_u32(pv_done + t), (j - 1) & 1, abort, kWaitNs);
+        if (!gate_ok) {
+          ok = mbar_wait(gate, gate_par, abort, kWaitNs);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
         }
         tc_fence_after();
+        s_ready = has_next;
+        if (grow && j > 0) {
+#pragma unroll
+          for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
+            uint32_t o[16];
+            tmem_ld16(tO + c0, o);
+            tmem_wait_ld();
+            reg_fence<16>(o);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st16(tO + c0, o);
+          }
+        }
         if (wq == 0 && lane == 0) PF_TRACE_AT(7, t, j);
         tmem_st32(tO + 64, pk);
         tmem_st32(tO + 96, pk + 32);
