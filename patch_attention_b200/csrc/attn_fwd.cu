@@ -92,7 +92,8 @@ constexpr int kThreads = 384;          // 3 warpgroups: softmax 0, softmax 1, MM
 constexpr uint32_t kRegsSoftmax = 208;
 constexpr uint32_t kRegsOther = 88;
 static_assert(128 * kRegsOther + 256 * kRegsSoftmax <= kThreads * 168, "register split");
-constexpr int kWarpMma = 8;
+constexpr int kWarpMma = 8;     // TMEM allocation; MMA issuer (of query tile 0 when split)
+constexpr int kWarpMma2 = 11;   // MMA issuer of query tile 1 on the separate-P layout
 constexpr int kWarpLoad = 9;
 constexpr int kWarpScatter = 10;
 constexpr uint32_t kTmemCols = 512;
@@ -312,6 +313,12 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
   // head_dim 64: O_t needs only 64 of its 128 TMEM columns, so P_t lives in the other 64
   // instead of over S_t, and the next QK need not wait for the current PV.
   constexpr bool kSepP = Dm::kMmaN <= 64;
+  // MMA issuing threads.  On the separate-P layout each query tile has its own (a
+  // tcgen05.mma holds its issuing thread for about its execution time, so one thread would
+  // make each tile's next QK wait behind the other tile's PV); on the P-over-S layout one
+  // thread issues for both tiles, which keeps the two softmax warpgroups staggered (two
+  // issuers measured slower there: both tiles' MMAs then contend in lockstep).
+  constexpr int kIssuers = kSepP ? NQ : 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -324,8 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
   uint64_t* s_full = kv_empty + S;
   uint64_t* p_full = s_full + 2;
   uint64_t* o_full = p_full + 2;
-  uint64_t* mma_done = o_full + 2;
-  uint64_t* s_free = mma_done + 1;   // separate-P layout: softmax has S in registers
+  uint64_t* mma_done = o_full + 2;   // [issuer]
+  uint64_t* s_free = mma_done + 2;   // separate-P layout: softmax has S in registers
   uint64_t* pv_done = s_free + 2;    // separate-P layout: PV of a tile has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -345,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
     mbar_init(smem_u32(q_full), 1);
     for (int s = 0; s < S; ++s) {
       mbar_init(smem_u32(kv_full + s), 1);
-      mbar_init(smem_u32(kv_empty + s), 1);
+      mbar_init(smem_u32(kv_empty + s), kIssuers);  // one commit per MMA issuer
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(smem_u32(s_full + t), 1);
@@ -353,6 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
       mbar_init(smem_u32(o_full + t), 1);
     }
     mbar_init(smem_u32(mma_done), 1);
+    mbar_init(smem_u32(mma_done + 1), 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(smem_u32(s_free + t), 4);  // one arrival per softmax warp
       mbar_init(smem_u32(pv_done + t), 1);
@@ -433,9 +441,10 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
       for (int i = issued > S ? issued - S : 0; i < issued; ++i)
         mbar_wait(smem_u32(kv_full + (i % S)), (i / S) & 1, nullptr, kWaitNs);
     }
-  } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == kWarpMma || (kIssuers == 2 && warp == kWarpMma2)) {
+    // ------------------------------------------------------------ MMA issuer(s)
     if (lane == 0) {
+      const int me = warp == kWarpMma ? 0 : 1;  // issuer index (the query tile, when split)
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, Dm::kMmaN, 1);
       const uint32_t q_base = smem_u32(sQ);
@@ -473,14 +482,13 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
         // P has its own TMEM columns: QK of the next key tile is issued as soon as the
         // softmax has S of the current one in registers, so the tensor core computes
         // S(j+1) while the softmax is still exponentiating tile j.
+        const int t = me;  // this issuer's query tile
         if (ok && n_tiles > 0) {
           ok = mbar_wait(smem_u32(kv_full + 0), 0, abort, kWaitNs);  // K(0): load 0, stage 0
           tc_fence_after();
           if (ok) {
-            for (int t = 0; t < NQ; ++t) {
-              issue_qk(t, 0);
-              mma_commit(smem_u32(s_full + t));
-            }
+            issue_qk(t, 0);
+            mma_commit(smem_u32(s_full + t));
             mma_commit(smem_u32(kv_empty + 0));
           }
         }
@@ -488,30 +496,22 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
           if (j + 1 < n_tiles) {
             const int iK = 2 * (j + 1), sK = iK % S;
             if (!(ok = mbar_wait(smem_u32(kv_full + sK), (iK / S) & 1, abort, kWaitNs))) break;
+            if (t == 0) PF_TRACE_AT(4, 0, j + 1);
+            if (!(ok = mbar_wait(smem_u32(s_free + t), j & 1, abort, kWaitNs))) break;
             tc_fence_after();
-            PF_TRACE_AT(4, 0, j + 1);
-            for (int t = 0; t < NQ; ++t) {
-              if (!(ok = mbar_wait(smem_u32(s_free + t), j & 1, abort, kWaitNs))) break;
-              tc_fence_after();
-              issue_qk(t, sK);
-              mma_commit(smem_u32(s_full + t));
-              PF_TRACE_AT(3, t, j + 1);
-            }
-            if (!ok) break;
+            issue_qk(t, sK);
+            mma_commit(smem_u32(s_full + t));
             mma_commit(smem_u32(kv_empty + sK));
+            PF_TRACE_AT(3, t, j + 1);
           }
           const int iV = 2 * j + 1, sV = iV % S;
           if (!(ok = mbar_wait(smem_u32(kv_full + sV), (iV / S) & 1, abort, kWaitNs))) break;
+          if (t == 0) PF_TRACE_AT(9, 0, j);
+          if (!(ok = mbar_wait(smem_u32(p_full + t), j & 1, abort, kWaitNs))) break;
           tc_fence_after();
-          PF_TRACE_AT(9, 0, j);
-          for (int t = 0; t < NQ; ++t) {
-            if (!(ok = mbar_wait(smem_u32(p_full + t), j & 1, abort, kWaitNs))) break;
-            tc_fence_after();
-            PF_TRACE_AT(2, t, j);
-            issue_pv(t, sV, j > 0);
-            mma_commit(smem_u32(pv_done + t));
-          }
-          if (!ok) break;
+          PF_TRACE_AT(2, t, j);
+          issue_pv(t, sV, j > 0);
+          mma_commit(smem_u32(pv_done + t));
           mma_commit(smem_u32(kv_empty + sV));
         }
       } else {
@@ -558,8 +558,8 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
       }
       if (!ok) raise_abort(abort, kWdMma);
       // drain every MMA issued by this thread before TMEM is released
-      mma_commit(smem_u32(mma_done));
-      mbar_wait(smem_u32(mma_done), 0, nullptr, kWaitNs);
+      mma_commit(smem_u32(mma_done + me));
+      mbar_wait(smem_u32(mma_done + me), 0, nullptr, kWaitNs);
     }
   } else if (warp == kWarpScatter) {
     // ------------------------------------------------------------ buffer scatter
