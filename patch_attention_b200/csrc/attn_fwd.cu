@@ -665,6 +665,9 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
         const float mxs = row_max128(s) * c;
         if (wq == 0 && lane == 0) PF_TRACE_AT(6, t, j);
         const bool grow = mxs > m + 8.f;
+        // the O rescale below uses warp-collective TMEM accesses: the whole warp takes it
+        // when any of its rows grew (alpha is exactly 1 for the others)
+        const bool any_grow = __any_sync(0xffffffffu, grow);
         const float alpha = grow ? ex2(m - mxs) : 1.f;
         l *= alpha;
         m = grow ? mxs : m;
@@ -699,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
         }
         tc_fence_after();
         s_ready = has_next;
-        if (grow && j > 0) {
+        if (any_grow && j > 0) {
 #pragma unroll
           for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
             uint32_t o[16];
@@ -729,7 +732,9 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
       bool exact = (j == 0) || (nv < kRows);
       if (!exact) {
         float xm = speculative_exps<kPolyPairs<D>>(s, c, m, pk, lsum);
-        if (xm > 8.f) {
+        // warp-uniform decision (the reload is a warp-collective TMEM access): if any row of
+        // the warp exceeded 2^8, the whole warp redoes the tile exactly
+        if (__any_sync(0xffffffffu, xm > 8.f)) {
           // S is still in TMEM (P has not been written yet): reload it for the exact path
           exact = true;
           tmem_ld32(tS + 0, s);
@@ -747,22 +752,22 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
             if (k >= nv) s[k] = __float_as_uint(-INFINITY);
         }
         const float mxs = row_max128(s) * c;
-        if (mxs > m + 8.f) {
-          const float alpha = ex2(m - mxs);
-          l *= alpha;
-          if (j > 0) {
+        const bool grow = mxs > m + 8.f;
+        const float alpha = grow ? ex2(m - mxs) : 1.f;
+        l *= alpha;
+        m = grow ? mxs : m;
+        // warp-collective TMEM accesses: the whole warp rescales when any row grew
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll
-            for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
-              uint32_t o[16];
-              tmem_ld16(tO + c0, o);
-              tmem_wait_ld();
-              reg_fence<16>(o);
+          for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
+            uint32_t o[16];
+            tmem_ld16(tO + c0, o);
+            tmem_wait_ld();
+            reg_fence<16>(o);
 #pragma unroll
-              for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-              tmem_st16(tO + c0, o);
-            }
+            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st16(tO + c0, o);
           }
-          m = mxs;
         }
         exact_exps(s, c, m, pk, lsum);
       }
