@@ -181,3 +181,12 @@ def test_workspace_sizes_and_checks():
         assert L.pf_set_workspace(None, FAKE, ws, None) == pa.PF_ERR_INVALID_ARG
     finally:
         pa.pf_destroy(ctx)
+
+
+def test_workspace_covers_the_text_query_call():
+    # 64-row patches but 512 text tokens: the text-query call has more query-tile groups than
+    # a patch call, and the workspace must hold its counters and partials too
+    few = _cfg(heads=8, n_img=1024, n_patches=16, n_txt=8, head_dim=128, n_layers=1)
+    many = _cfg(heads=8, n_img=1024, n_patches=16, n_txt=512, head_dim=128, n_layers=1)
+    assert pa.pf_workspace_bytes(many) > pa.pf_workspace_bytes(few) > 0
+
