@@ -10,12 +10,16 @@
 // Design (per CTA = one head of one batch element, NQ x 128 query rows):
 //   warps 0-3 / 4-7  softmax for query tile 0 / 1: one thread owns one query row (one
 //                    TMEM lane), so the row max and row sum need no shuffles.
-//   warp 8           TMEM allocation and the single-thread tcgen05.mma issuer.
+//   warp 8           TMEM allocation and a single-thread tcgen05.mma issuer (of both
+//                    query tiles, or of tile 0 on the separate-P layout).
 //   warp 9           TMA producer: Q tiles once, then K/V tiles through a smem ring.
 //   warp 10          scatter of the CTA's share of K_p/V_p into the buffer.
-// S = Q K^T lands in TMEM (fp32, 128 columns per query tile); the softmax overwrites its
-// first 64 columns with P as packed bf16, which the PV MMA reads straight from TMEM
-// (A operand in TMEM, V as an MN-major B operand in smem).  O accumulates in TMEM.
+//   warp 11          separate-P layout only: the MMA issuer of query tile 1.
+// S = Q K^T lands in TMEM (fp32, 128 columns per query tile); P (packed bf16) is written
+// over S's first 64 columns, or, when head_dim is 64, into the free half of O's columns
+// (the separate-P layout, so the next QK overlaps the softmax).  The PV MMA reads P
+// straight from TMEM (A operand in TMEM, V as an MN-major B operand in smem).  O
+// accumulates in TMEM.
 // The context is walked as segments so that patch p's rows are read from the fresh
 // tensors, never from buffer rows that other CTAs of this launch are writing:
 //   [fresh rows 0..P) | buffer rows 0..pP) | buffer rows (p+1)P..N) | text rows 0..T)
