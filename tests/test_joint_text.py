@@ -63,13 +63,14 @@ def test_host_argument_checks():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("d,T", [(64, 154), (72, 120), (128, 512), (128, 40), (64, 300)])
+@pytest.mark.parametrize("d,T,B", [(64, 154, 1), (72, 120, 1), (128, 512, 1), (128, 40, 1),
+                                   (64, 300, 1), (128, 154, 2)])
 @pytest.mark.parametrize("schedule", [pa.PF_SCHED_PIPEFUSION, pa.PF_SCHED_DISTRIFUSION])
-def test_text_queries_against_buffer_and_text(d, T, schedule):
-    wl = synth.AttnWorkload("txt", 1, 3, d, 24, 32, 4, T, 1, 2, 0.95, 0.3)
+def test_text_queries_against_buffer_and_text(d, T, B, schedule):
+    wl = synth.AttnWorkload("txt", B, 3, d, 24, 32, 4, T, 1, 2, 0.95, 0.3)
     P = wl.patch_len
     gen = synth.AttnInputs(wl, seed=7, device="cuda")
-    pat = pa.PatchAttention(1, 3, d, wl.n_img, 4, T, 1, schedule=schedule)
+    pat = pa.PatchAttention(B, 3, d, wl.n_img, 4, T, 1, schedule=schedule)
     g = torch.Generator(device="cuda").manual_seed(11)
     try:
         prev = None
@@ -78,7 +79,7 @@ def test_text_queries_against_buffer_and_text(d, T, schedule):
             if s == 0:
                 pat.init_layer(0, cur["k"], cur["v"])
                 prev = cur
-            q_txt = torch.randn(1, T, 3, d, device="cuda", generator=g).bfloat16()
+            q_txt = torch.randn(B, T, 3, d, device="cuda", generator=g).bfloat16()
             for p in range(4):
                 sl = slice(p * P, (p + 1) * P)
                 pat.step(0, p, cur["q"][:, sl].contiguous(), cur["k"][:, sl].contiguous(),
@@ -87,19 +88,24 @@ def test_text_queries_against_buffer_and_text(d, T, schedule):
                     # mid-step: the buffer holds this step for patches <= 1 under PipeFusion,
                     # the previous step everywhere under DistriFusion
                     o = pat.text_step(0, q_txt, cur["k_txt"], cur["v_txt"])
-                    if schedule == pa.PF_SCHED_PIPEFUSION:
-                        kb = oracle.expected_buffer(f64(cur["k"][0]), f64(prev["k"][0]), 1, 4)
-                        vb = oracle.expected_buffer(f64(cur["v"][0]), f64(prev["v"][0]), 1, 4)
-                    else:
-                        kb, vb = f64(prev["k"][0]), f64(prev["v"][0])
-                    ref = oracle.attend(f64(q_txt[0]), np.concatenate([kb, f64(cur["k_txt"][0])]),
-                                        np.concatenate([vb, f64(cur["v_txt"][0])]), wl.softmax_scale)
-                    _close(f64(o[0]), ref, f64(cur["v"][0]), f64(prev["v"][0]), f64(cur["v_txt"][0]))
+                    for bi in range(B):
+                        if schedule == pa.PF_SCHED_PIPEFUSION:
+                            kb = oracle.expected_buffer(f64(cur["k"][bi]), f64(prev["k"][bi]), 1, 4)
+                            vb = oracle.expected_buffer(f64(cur["v"][bi]), f64(prev["v"][bi]), 1, 4)
+                        else:
+                            kb, vb = f64(prev["k"][bi]), f64(prev["v"][bi])
+                        ref = oracle.attend(f64(q_txt[bi]), np.concatenate([kb, f64(cur["k_txt"][bi])]),
+                                            np.concatenate([vb, f64(cur["v_txt"][bi])]), wl.softmax_scale)
+                        _close(f64(o[bi]), ref, f64(cur["v"][bi]), f64(prev["v"][bi]),
+                               f64(cur["v_txt"][bi]))
             # after the step: the buffer is all this step's K/V
             o = pat.text_step(0, q_txt, cur["k_txt"], cur["v_txt"])
-            ref = oracle.attend(f64(q_txt[0]), np.concatenate([f64(cur["k"][0]), f64(cur["k_txt"][0])]),
-                                np.concatenate([f64(cur["v"][0]), f64(cur["v_txt"][0])]), wl.softmax_scale)
-            _close(f64(o[0]), ref, f64(cur["v"][0]), f64(cur["v_txt"][0]))
+            for bi in range(B):
+                ref = oracle.attend(f64(q_txt[bi]),
+                                    np.concatenate([f64(cur["k"][bi]), f64(cur["k_txt"][bi])]),
+                                    np.concatenate([f64(cur["v"][bi]), f64(cur["v_txt"][bi])]),
+                                    wl.softmax_scale)
+                _close(f64(o[bi]), ref, f64(cur["v"][bi]), f64(cur["v_txt"][bi]))
             assert pat.next_patch(0) == 0
             prev = cur
         pat.check()
