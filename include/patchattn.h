@@ -233,6 +233,16 @@ pf_status pf_switch_update(pf_switch* s, float relmae, int* phase_out);
  * stream reported an error, else PF_OK. */
 pf_status pf_check_device_status(pf_ctx* ctx, void* stream);
 
+/* Self-test of failure detection (the pages have no counterpart): launches a one-thread
+ * kernel whose mbarrier wait is never satisfied, so its bounded wait gives up after
+ * limit_ns (1 ns .. 10 s), sets its bit in the device status word and returns -- the path
+ * every role of the attention kernel takes when a wait expires, without faulting or hanging
+ * the device.  Synchronises `stream`, then reads and clears the status word.  Returns
+ * PF_ERR_TIMEOUT when the wait gave up as designed (PF_OK would mean it did not), PF_ERR_CUDA
+ * on a CUDA error, PF_ERR_INVALID_ARG for a limit out of range.  Shares the status word with
+ * the other kernels: do not run it while attention launches are in flight. */
+pf_status pf_selftest_bounded_wait(uint64_t limit_ns, void* stream);
+
 /* Static description of a status code (never NULL). */
 const char* pf_status_string(pf_status s);
 

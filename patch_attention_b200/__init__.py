@@ -36,7 +36,7 @@ EXPORTED = [
     "pf_kvbuf_bytes", "pf_create", "pf_destroy", "pf_kvbuf_init", "pf_patch_attn_step",
     "pf_get_state", "pf_set_state", "pf_workspace_bytes", "pf_set_workspace",
     "pf_cfg_workspace_bytes", "pf_cfg_combine_relmae", "pf_cfg_combine_relmae_static",
-    "pf_check_device_status", "pf_status_string", "pf_version", "pf_switch_init",
+    "pf_check_device_status", "pf_selftest_bounded_wait", "pf_status_string", "pf_version", "pf_switch_init",
     "pf_switch_update", "pf_text_attn_step", "pf_qk_rmsnorm",
 ]
 
@@ -94,6 +94,7 @@ def _lib():
             "pf_cfg_combine_relmae": (i, [vp, vp, i, i64, f, vp, vp, vp, vp, sz, vp]),
             "pf_cfg_combine_relmae_static": (i, [vp, vp, i, i64, f, vp, vp, vp, vp]),
             "pf_check_device_status": (i, [vp, vp]),
+            "pf_selftest_bounded_wait": (i, [ctypes.c_uint64, vp]),
             "pf_status_string": (ctypes.c_char_p, [i]),
             "pf_text_attn_step": (i, [vp, i, vp, vp, vp, vp, vp]),
             "pf_qk_rmsnorm": (i, [vp, i64, i, vp, f, vp]),
@@ -292,6 +293,11 @@ class HybridCfgSwitch:
 
 def pf_check_device_status(ctx, stream=None) -> None:
     _check(_lib().pf_check_device_status(ctx, _stream(stream)), "pf_check_device_status")
+
+
+def pf_selftest_bounded_wait(limit_ns: int, stream=None) -> int:
+    """Run the failure-detection self-test; returns the status (PF_ERR_TIMEOUT as designed)."""
+    return int(_lib().pf_selftest_bounded_wait(int(limit_ns), _stream(stream)))
 
 
 # ------------------------------------------------------------------ convenience

@@ -105,7 +105,7 @@ constexpr uint32_t kColO = 256;        // O_t at column 256 + 128 t; S_t at colu
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kMaxSplit = 16;          // most key-range parts per query tile
 
-enum : unsigned { kWdLoad = 1u, kWdMma = 2u, kWdSoftmax = 4u, kWdEpilogue = 8u };
+enum : unsigned { kWdLoad = 1u, kWdMma = 2u, kWdSoftmax = 4u, kWdEpilogue = 8u, kWdSelftest = 16u };
 
 template <int D>
 struct Dims {
@@ -989,6 +989,25 @@ extern "C" int pf_trace_cta_read(unsigned long long* dst, size_t n) {
   return static_cast<int>(cudaMemcpyFromSymbol(dst, g_cta, n * sizeof(unsigned long long)));
 }
 #endif
+
+namespace {
+// One thread waits on an mbarrier that nothing ever arrives at.  The wait gives up after
+// limit_ns and records the role in the status word: the path every role of the attention
+// kernel takes when one of its bounded waits expires.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+    if (!mbar_wait(smem_u32(&bar), 0, nullptr, limit_ns)) atomicOr(&g_watchdog, kWdSelftest);
+  }
+}
+}  // namespace
+
+cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream) {
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(static_cast<unsigned long long>(limit_ns));
+  return cudaGetLastError();
+}
 
 cudaError_t read_and_clear_watchdog(unsigned* value) {
   unsigned v = 0;

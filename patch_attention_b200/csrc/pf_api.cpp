@@ -476,6 +476,16 @@ pf_status pf_check_device_status(pf_ctx* ctx, void* stream) {
   return v ? PF_ERR_TIMEOUT : PF_OK;
 }
 
+pf_status pf_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return PF_ERR_INVALID_ARG;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (pf::launch_selftest_wait(limit_ns, st) != cudaSuccess) return PF_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PF_ERR_CUDA;
+  unsigned v = 0;
+  if (pf::read_and_clear_watchdog(&v) != cudaSuccess) return PF_ERR_CUDA;
+  return v ? PF_ERR_TIMEOUT : PF_OK;
+}
+
 const char* pf_status_string(pf_status s) {
   switch (s) {
     case PF_OK: return "ok";

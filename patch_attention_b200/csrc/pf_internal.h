@@ -81,6 +81,10 @@ int cfg_static_capacity_samples();
 // Device word written by kernels whose bounded waits expired (0 = none).
 cudaError_t read_and_clear_watchdog(unsigned* value);
 
+// A one-thread kernel whose bounded wait can never be satisfied: it gives up after limit_ns
+// and sets its bit in the device word above.
+cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream);
+
 // Host check that a device of compute capability 10.x is current.
 bool device_is_sm100();
 

@@ -190,3 +190,9 @@ def test_workspace_covers_the_text_query_call():
     many = _cfg(heads=8, n_img=1024, n_patches=16, n_txt=512, head_dim=128, n_layers=1)
     assert pa.pf_workspace_bytes(many) > pa.pf_workspace_bytes(few) > 0
 
+
+def test_selftest_rejects_limits_out_of_range():
+    L = pa._lib()
+    assert L.pf_selftest_bounded_wait(0, None) == pa.PF_ERR_INVALID_ARG
+    assert L.pf_selftest_bounded_wait(10_000_000_001, None) == pa.PF_ERR_INVALID_ARG
+
