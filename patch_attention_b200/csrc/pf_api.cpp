@@ -54,11 +54,6 @@ EncodeTiledFn encode_fn() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool config_ok(const pf_config* c) {
-  return c && c->batch >= 1 && c->heads >= 1 && c->n_img >= 1 && c->n_patches >= 1 &&
-         c->n_txt >= 0 && c->n_layers >= 1;
-}
-
 pf_status check_config(const pf_config* c) {
   if (!c) return PF_ERR_INVALID_ARG;
   if (c->batch < 1 || c->heads < 1 || c->n_img < 1 || c->n_patches < 1 || c->n_txt < 0 ||
