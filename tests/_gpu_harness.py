@@ -2,8 +2,7 @@
 C ABI (via the Python binding) and compares against the fp64 oracle."""
 from __future__ import annotations
 
-import math
-from typing import Iterable, Optional
+from typing import Optional
 
 import numpy as np
 import torch

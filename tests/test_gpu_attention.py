@@ -13,7 +13,7 @@ import torch
 import oracle
 import patch_attention_b200 as pa
 from patch_attention_b200 import synth
-from tests._gpu_harness import Checker, f64, run_workload
+from tests._gpu_harness import f64, run_workload
 
 pytestmark = pytest.mark.gpu
 

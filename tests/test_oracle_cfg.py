@@ -4,7 +4,6 @@ import math
 import os
 
 import numpy as np
-import torch
 
 import oracle
 from patch_attention_b200 import synth
