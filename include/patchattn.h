@@ -82,7 +82,9 @@ typedef struct {
 typedef struct pf_ctx pf_ctx; /* opaque, host-only */
 
 /* Bytes of ONE layer's K/V buffer: K region [B, N, H, d] bf16 followed by the V region of
- * the same size (2 * B * N * H * d * 2 bytes).  0 if cfg is NULL or invalid. */
+ * the same size (2 * B * N * H * d * 2 bytes); under PF_SCHED_DISTRIFUSION a second such
+ * [K | V] half follows (the step being written while the other half is read), twice the
+ * bytes.  0 if cfg is NULL or invalid. */
 size_t pf_kvbuf_bytes(const pf_config* cfg);
 
 /* Create a context.  kvbuf_per_layer: host array of n_layers device pointers, each to a
@@ -103,11 +105,15 @@ pf_status pf_kvbuf_init(pf_ctx* ctx, int layer, const void* k_full, const void* 
  *   q_p, k_p, v_p : fresh activations of the patch, [B, P, H, d] bf16
  *   k_txt, v_txt  : this step's text keys/values, [B, T, H, d] bf16 (both NULL iff T == 0)
  *   o_p           : output, [B, P, H, d] bf16, o_p = softmax(scale Q_p [K';K_txt]^T) [V';V_txt]
- *                   where K', V' is the buffer with patch p's rows replaced by k_p, v_p.
- * Under PF_SCHED_PIPEFUSION the call also writes k_p, v_p into the buffer rows of patch p
- * (fused into the attention kernel); o_p must not alias any input.
+ *                   where K', V' is the buffer being read with patch p's rows replaced by
+ *                   k_p, v_p.
+ * The call also writes k_p, v_p into the buffer rows of patch p, fused into the attention
+ * kernel: under PF_SCHED_PIPEFUSION into the buffer it reads (later patches of the step see
+ * them), under PF_SCHED_DISTRIFUSION into the other half, which becomes the half read once
+ * all M patches of the step have been called.  o_p must not alias any input.
  * Errors: PF_ERR_STATE before pf_kvbuf_init(layer); PF_ERR_ORDER if `patch` is not the
- * layer's next patch; PF_ERR_INVALID_ARG / PF_ERR_ALIGN for bad pointers. */
+ * layer's next patch (PipeFusion) or was already called this step (DistriFusion);
+ * PF_ERR_INVALID_ARG / PF_ERR_ALIGN for bad pointers. */
 pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
                              const void* k_p, const void* v_p, const void* k_txt,
                              const void* v_txt, void* o_p, void* stream);
