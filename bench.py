@@ -19,6 +19,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -247,120 +248,257 @@ def run_reference(args, world, rank):
 
 # ----------------------------------------------------------------------------------- GPU
 
+L2_BYTES = 126 << 20
+NOMINAL_FLOP_PER_CLK_SM = 8192  # dense bf16 tcgen05: one 128x128x16 MMA per 64 cycles per SM
+
+
+def n_sms(dev) -> int:
+    return torch.cuda.get_device_properties(dev).multi_processor_count
+
+
+class StepRunner:
+    """One attention workload resident in HBM: per-layer buffers, `n_sets` alternating input
+    sets (AR(1) steps) and outputs.  A step = every patch in order x every layer through
+    pf_patch_attn_step, then one guidance combine over the model's latent."""
+
+    def __init__(self, pa, wl, dev, seed, min_set_bytes=2 * L2_BYTES):
+        self.pa, self.wl, self.dev = pa, wl, dev
+        B, H, d, N, M, T, L = wl.batch, wl.heads, wl.head_dim, wl.n_img, wl.n_patches, wl.n_txt, wl.n_layers
+        assert B == 1, "patch slices are passed as views; batch 1 keeps them contiguous"
+        set_bytes = L * (3 * N + 2 * T) * H * d * 2
+        # enough alternating input sets that consecutive steps' inputs together exceed L2
+        self.n_sets = max(2, -(-min_set_bytes // set_bytes))
+        gen = synth.AttnInputs(wl, seed=seed, device=dev)
+        self.sets = [[gen.step_tensors(l) for l in range(L)] for _ in range(self.n_sets)]
+        del gen  # drop the fp32 AR(1) state
+        torch.cuda.empty_cache()
+        self.set_bytes = set_bytes
+        self.pat = pa.PatchAttention(B, H, d, N, M, T, L)
+        for l in range(L):
+            self.pat.init_layer(l, self.sets[0][l]["k"], self.sets[0][l]["v"])
+        self.outs = [torch.empty(B, N, H, d, dtype=torch.bfloat16, device=dev) for _ in range(L)]
+        self.cshape = CFG_SHAPE[wl.name]
+        self.cwl = synth.CfgWorkload("cfg", B, *self.cshape)
+        self.c_in, self.u_in = synth.CfgInputs(self.cwl, device=dev).step_tensors(25)
+        self.n_cfg = self.c_in.numel() // B
+        self.cfg_out = torch.empty(self.c_in.shape, dtype=torch.bfloat16, device=dev)
+        self.rel = torch.empty(B, dtype=torch.float32, device=dev)
+        self.cws = torch.empty(max(16, pa.pf_cfg_workspace_bytes(B, self.n_cfg)), dtype=torch.uint8, device=dev)
+        self.L_ = pa._lib()
+        self.row_bytes = H * d * 2
+        # precomputed pointers: the timed loop is argument marshalling only
+        self.ptrs = []
+        for st in range(self.n_sets):
+            per = []
+            for l in range(L):
+                t = self.sets[st][l]
+                per.append((t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(),
+                            t["k_txt"].data_ptr() if T else None, t["v_txt"].data_ptr() if T else None))
+            self.ptrs.append(per)
+        self.optrs = [o.data_ptr() for o in self.outs]
+        self.launches_per_step = M * L + 2  # attention launches + guidance partial + finalize
+
+    def attn_section(self, set_idx, sh):
+        wl, L_, ctx = self.wl, self.L_, self.pat.ctx
+        per = self.ptrs[set_idx % self.n_sets]
+        for p in range(wl.n_patches):
+            off = p * wl.patch_len * self.row_bytes
+            for l in range(wl.n_layers):
+                q, k, v, kt, vt = per[l]
+                st = L_.pf_patch_attn_step(ctx, l, p, q + off, k + off, v + off, kt, vt, self.optrs[l] + off, sh)
+                if st != 0:
+                    raise self.pa.PatchAttnError(st, "pf_patch_attn_step")
+
+    def cfg_section(self, sh):
+        st = self.L_.pf_cfg_combine_relmae(self.c_in.data_ptr(), self.u_in.data_ptr(), self.wl.batch, self.n_cfg,
+                                           self.cwl.w, None, self.cfg_out.data_ptr(), self.rel.data_ptr(),
+                                           self.cws.data_ptr(), self.cws.numel(), sh)
+        if st != 0:
+            raise self.pa.PatchAttnError(st, "pf_cfg_combine_relmae")
+
+    def run(self, steps, first_set, world, sample_clocks=True):
+        """Time exactly `steps` steps (barrier + synchronize on both sides).  Returns the
+        total ms, per-step attention and guidance ms from events on the launching stream,
+        and the clock samples taken during the timed region."""
+        dev = self.dev
+        stream = torch.cuda.current_stream(dev)
+        sh = stream.cuda_stream
+        ev = lambda: torch.cuda.Event(enable_timing=True)
+        a0 = [ev() for _ in range(steps)]
+        a1 = [ev() for _ in range(steps)]
+        c1 = [ev() for _ in range(steps)]
+        start, stop = ev(), ev()
+        clocks = ClockSampler(dev.index or 0) if sample_clocks else None
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        if clocks:
+            clocks.start()
+            time.sleep(0.3)  # let the sampler attach before the timed region
+        start.record(stream)
+        for i in range(steps):
+            a0[i].record(stream)
+            self.attn_section(first_set + i, sh)
+            a1[i].record(stream)
+            self.cfg_section(sh)
+            c1[i].record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+        clock_info = clocks.stop() if clocks else None
+        barrier(world)
+        self.pat.check()
+        total = start.elapsed_time(stop)
+        attn = sum(a0[i].elapsed_time(a1[i]) for i in range(steps)) / steps
+        cfg = sum(a1[i].elapsed_time(c1[i]) for i in range(steps)) / steps
+        return total, attn, cfg, clock_info
+
+    def warm(self, steps):
+        sh = torch.cuda.current_stream(self.dev).cuda_stream
+        for i in range(steps):
+            self.attn_section(i + 1, sh)
+            self.cfg_section(sh)
+        torch.cuda.synchronize(self.dev)
+        self.pat.check()
+
+    def close(self):
+        self.pat.close()
+
+
+def per_clock(tflops, clock_info, sms):
+    """FLOP per SM per clock at the median SM clock of the timed region, and its fraction
+    of the nominal dense bf16 rate (8192 FLOP/clk/SM)."""
+    if not clock_info or not clock_info.get("sm_mhz"):
+        return None, None
+    f = tflops * 1e12 / (sms * clock_info["sm_mhz"] * 1e6)
+    return f, f / NOMINAL_FLOP_PER_CLK_SM
+
+
+def attn_roofline(wl, attn_ms, timed_s, peaks, peak_src, clock_info, sms, traffic):
+    """Roofline of patch_attn_kernel: algorithmic FLOP per launch / average launch time
+    (events around each step's attention section, launch gaps included).  The peak is the
+    measured sustained bf16 rate when the timed region lasts at least 2 s, else the burst."""
+    launch_ms = attn_ms / (wl.n_patches * wl.n_layers)
+    achieved = wl.flop_per_call() / (launch_ms * 1e-3) / 1e12
+    sustained = timed_s >= 2.0
+    key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    peak = float(peaks.get(key, peaks.get("bf16_tflops")))
+    fpc, fpc_frac = per_clock(achieved, clock_info, sms)
+    return {"bound": "tensor", "kernel": "patch_attn_kernel", "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+            "peak_source": f"{peak_src} {key} ({'timed region >= 2 s' if sustained else 'timed region < 2 s'})",
+            "launch_ms": launch_ms, "flop_per_launch": wl.flop_per_call(),
+            "flop_per_clk_sm": fpc, "frac_of_nominal_per_clk": fpc_frac}
+
+
+def sub_record(pa, name, dev, seed, world, peaks, peak_src, min_timed_s=2.0, max_steps=20000):
+    """A workload other than the headline, timed over at least `min_timed_s` of steps so that
+    the sustained peak is the right denominator; its own clock samples."""
+    wl = synth.ATTN_WORKLOADS[name]
+    r = StepRunner(pa, wl, dev, seed if seed is not None else synth.default_seed(name))
+    try:
+        r.warm(3)
+        total, _, _, _ = r.run(3, 4, 1, sample_clocks=False)
+        t_step = total / 3 / 1e3
+        steps = int(min(max_steps, max(20, math.ceil(min_timed_s * 1.1 / t_step))))
+        steps = int(max_over_ranks(float(steps), world))  # every rank times the same count
+        total, attn, cfg, clk = r.run(steps, 7, world)
+    finally:
+        r.close()
+    ms = max_over_ranks(total / steps, world)
+    flop_step = wl.n_layers * wl.flop_per_layer_step()
+    value = world * flop_step / (ms * 1e-3) / 1e12
+    sms = n_sms(dev)
+    rec = {"workload": name, "steps": steps, "timed_s": total / 1e3, "ms_per_step": ms,
+           "value": value, "unit": "TFLOP/s", "attn_ms_per_step": attn, "cfg_ms_per_step": cfg,
+           "flop_per_step": flop_step,
+           "config": {"heads": wl.heads, "head_dim": wl.head_dim, "n_img": wl.n_img,
+                      "n_patches": wl.n_patches, "patch_len": wl.patch_len, "n_txt": wl.n_txt,
+                      "layers": wl.n_layers},
+           "l2": f"{r.n_sets} alternating input sets of {r.set_bytes / 1e6:.0f} MB (together > 2x L2)",
+           "roofline": attn_roofline(wl, attn, total / 1e3, peaks, peak_src, clk, sms, load_traffic(name)),
+           "clocks": clk}
+    return rec
+
+
+def measure_copy_kernels(pa, r: StepRunner, hbm, reps=5):
+    """The start-up pass (pf_kvbuf_init) of one layer and the per-head RMS normalisation of a
+    full-spatial Q, both HBM bound and both larger than L2; median of `reps` calls."""
+    wl, dev = r.wl, r.dev
+    stream = torch.cuda.current_stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def timed(fn):
+        ts = []
+        for i in range(reps + 2):
+            e0, e1 = ev(), ev()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if i >= 2:
+                ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    t = r.sets[0][0]
+    init_ms = timed(lambda: r.pat.init_layer(0, t["k"], t["v"]))
+    init_bytes = 2 * 2 * t["k"].numel() * 2  # K and V, read + written
+    x = t["q"].clone()
+    norm_ms = timed(lambda: pa.pf_qk_rmsnorm(x))
+    norm_bytes = 2 * x.numel() * 2
+    del x
+    return {
+        "kvbuf_init": {"gb_per_s": init_bytes / (init_ms * 1e-3) / 1e9,
+                       "frac_hbm": init_bytes / (init_ms * 1e-3) / 1e9 / hbm, "ms": init_ms,
+                       "bytes": init_bytes, "what": f"one {wl.name} layer: K and V [1,{wl.n_img},{wl.heads},{wl.head_dim}] bf16 copied into the buffer"},
+        "qk_rmsnorm": {"gb_per_s": norm_bytes / (norm_ms * 1e-3) / 1e9,
+                       "frac_hbm": norm_bytes / (norm_ms * 1e-3) / 1e9 / hbm, "ms": norm_ms,
+                       "bytes": norm_bytes, "what": f"in place on a full-spatial {wl.name} Q [1,{wl.n_img},{wl.heads},{wl.head_dim}] bf16"},
+    }
+
+
+def scatter_record(wl, traffic):
+    """The fresh-K/V scatter is fused into the attention launch: its algorithmic bytes per
+    call (K_p and V_p read and written), and their share of the launch's DRAM traffic."""
+    b = 2 * 2 * wl.batch * wl.patch_len * wl.heads * wl.head_dim * 2
+    rec = {"bytes_per_call": b, "fused_into": "patch_attn_kernel",
+           "launch_dram_bytes": traffic, "share_of_launch_dram": (b / traffic) if traffic else None}
+    return rec
+
 
 def run_gpu(args, world, rank, local):
     import patch_attention_b200 as pa
 
     dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    sms = n_sms(dev)
     wl = synth.ATTN_WORKLOADS[args.workload]
-    B, H, d, N, M, T, L = wl.batch, wl.heads, wl.head_dim, wl.n_img, wl.n_patches, wl.n_txt, wl.n_layers
-    P = wl.patch_len
-    assert B == 1, "patch slices are passed as views; batch 1 keeps them contiguous"
+    r = StepRunner(pa, wl, dev, args.seed if args.seed is not None else synth.default_seed(wl.name))
+    r.warm(args.warmup)
+    total_ms, attn_ms, cfg_ms, clock_info = r.run(args.steps, args.warmup + 1, world)
 
-    # two input sets so consecutive steps see different activations (AR(1) steps)
-    gen = synth.AttnInputs(wl, seed=args.seed, device=dev)
-    sets = [[gen.step_tensors(l) for l in range(L)] for _ in range(2)]
-    del gen  # drop the fp32 AR(1) state
-    torch.cuda.empty_cache()
-    pat = pa.PatchAttention(B, H, d, N, M, T, L)
-    for l in range(L):
-        pat.init_layer(l, sets[0][l]["k"], sets[0][l]["v"])
-    outs = [torch.empty(B, N, H, d, dtype=torch.bfloat16, device=dev) for _ in range(L)]
-
-    cshape = CFG_SHAPE[wl.name]
-    cwl = synth.CfgWorkload("cfg", B, *cshape)
-    c_in, u_in = synth.CfgInputs(cwl, device=dev).step_tensors(25)
-    n_cfg = c_in.numel() // B
-    cfg_out = torch.empty(c_in.shape, dtype=torch.bfloat16, device=dev)
-    rel = torch.empty(B, dtype=torch.float32, device=dev)
-    ws = torch.empty(max(16, pa.pf_cfg_workspace_bytes(B, n_cfg)), dtype=torch.uint8, device=dev)
-
-    L_ = pa._lib()
-    ctx = pat.ctx
-    stream = torch.cuda.current_stream(dev)
-    sh = stream.cuda_stream
-    row_bytes = H * d * 2
-
-    # precomputed pointers: the timed loop is argument marshalling only
-    ptrs = []
-    for s in range(2):
-        per = []
-        for l in range(L):
-            t = sets[s][l]
-            per.append((t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(),
-                        t["k_txt"].data_ptr() if T else None, t["v_txt"].data_ptr() if T else None))
-        ptrs.append(per)
-    optrs = [o.data_ptr() for o in outs]
-
-    def attn_section(set_idx):
-        per = ptrs[set_idx]
-        for p in range(M):
-            off = p * P * row_bytes
-            for l in range(L):
-                q, k, v, kt, vt = per[l]
-                st = L_.pf_patch_attn_step(ctx, l, p, q + off, k + off, v + off, kt, vt, optrs[l] + off, sh)
-                if st != 0:
-                    raise pa.PatchAttnError(st, "pf_patch_attn_step")
-
-    def cfg_section():
-        st = L_.pf_cfg_combine_relmae(c_in.data_ptr(), u_in.data_ptr(), B, n_cfg, cwl.w, None,
-                                      cfg_out.data_ptr(), rel.data_ptr(), ws.data_ptr(), ws.numel(), sh)
-        if st != 0:
-            raise pa.PatchAttnError(st, "pf_cfg_combine_relmae")
-
-    ev = lambda: torch.cuda.Event(enable_timing=True)
-    launches_per_step = M * L + 2
-
-    # warm-up (the first step also validates the whole path)
-    for i in range(args.warmup):
-        attn_section((i + 1) % 2)
-        cfg_section()
-    torch.cuda.synchronize(dev)
-    pat.check()
-
-    a0 = [ev() for _ in range(args.steps)]
-    a1 = [ev() for _ in range(args.steps)]
-    c1 = [ev() for _ in range(args.steps)]
-    start, stop = ev(), ev()
-    clocks = ClockSampler(local)
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    clocks.start()
-    time.sleep(0.3)  # let the sampler attach before the timed region
-    start.record(stream)
-    for i in range(args.steps):
-        a0[i].record(stream)
-        attn_section((args.warmup + i + 1) % 2)
-        a1[i].record(stream)
-        cfg_section()
-        c1[i].record(stream)
-    stop.record(stream)
-    torch.cuda.synchronize(dev)
-    clock_info = clocks.stop()
-    barrier(world)
-    pat.check()
-
-    total_ms = start.elapsed_time(stop)
     ms_step = max_over_ranks(total_ms / args.steps, world)
-    attn_ms = sum(a0[i].elapsed_time(a1[i]) for i in range(args.steps)) / args.steps
-    cfg_ms = sum(a1[i].elapsed_time(c1[i]) for i in range(args.steps)) / args.steps
+    L, M, P = wl.n_layers, wl.n_patches, wl.patch_len
     flop_step = L * wl.flop_per_layer_step()
     value = world * flop_step / (ms_step * 1e-3) / 1e12
-
-    peaks, peak_src = load_peaks()
-    launch_ms = attn_ms / (M * L)
-    achieved = wl.flop_per_call() / (launch_ms * 1e-3) / 1e12
-    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     traffic = load_traffic(wl.name)
-    cfg_bytes = B * n_cfg * (4 + 4 + 2)
+    roof = attn_roofline(wl, attn_ms, total_ms / 1e3, peaks, peak_src, clock_info, sms, traffic)
+    cfg_bytes = wl.batch * r.n_cfg * (4 + 4 + 2)
     cfg_gbs = cfg_bytes / (cfg_ms * 1e-3) / 1e9
-    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
 
     cfg_big = measure_cfg_largest(pa, dev, hbm)
-
+    copies = measure_copy_kernels(pa, r, hbm)
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, world, local, wl, sets, pat, outs, c_in, u_in, cfg_out, rel, ws, cwl, n_cfg)
+        e2e = run_e2e(args, world, r)
+    r.close()
+    del r
+    torch.cuda.empty_cache()
+
+    subs = {}
+    if not args.no_sub:
+        for name in ("sd3", "pixart"):
+            if name != wl.name:
+                subs[name] = sub_record(pa, name, dev, None, world, peaks, peak_src)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -371,30 +509,31 @@ def run_gpu(args, world, rank, local):
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "batch": B, "heads": H, "head_dim": d, "n_img": N,
-                   "n_patches": M, "patch_len": P, "n_txt": T, "layers": L,
+        "config": {"workload": wl.name, "batch": wl.batch, "heads": wl.heads, "head_dim": wl.head_dim,
+                   "n_img": wl.n_img, "n_patches": M, "patch_len": P, "n_txt": wl.n_txt, "layers": L,
                    "calls_per_step": M * L, "flop_per_step": flop_step,
-                   "cfg_latent": list(cshape), "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2 (two alternating input sets of "
-                         f"{2 * L * 3 * N * H * d * 2 / 1e9:.1f} GB)"},
-        "pct_bf16_peak": 100.0 * value / world / peak,
-        "roofline": {"bound": "tensor", "kernel": "patch_attn_kernel", "achieved": achieved,
-                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "traffic": traffic,
-                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)"},
+                   "cfg_latent": list(CFG_SHAPE[wl.name]), "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (alternating input sets of "
+                         f"{(3 * wl.n_img + 2 * wl.n_txt) * wl.heads * wl.head_dim * 2 * L / 1e9:.1f} GB)"},
+        "pct_bf16_peak": 100.0 * value / world / roof["peak"],
+        "roofline": roof,
         "cfg_combine": {"in_step": {"gb_per_s": cfg_gbs, "frac_hbm": cfg_gbs / hbm, "ms": cfg_ms,
-                                    "bytes": cfg_bytes, "latent": [B] + list(cshape)},
+                                    "bytes": cfg_bytes, "latent": [wl.batch] + list(CFG_SHAPE[wl.name])},
                         "largest": cfg_big, "peak_gbs": hbm,
                         "peak_source": f"{peak_src} hbm_gbs"},
+        "kvbuf_init": copies["kvbuf_init"],
+        "scatter": scatter_record(wl, traffic),
+        "qk_rmsnorm": copies["qk_rmsnorm"],
+        "hbm_peak_gbs": hbm,
         "attn_ms_per_step": attn_ms,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": (M * L + 2) * args.steps,
         "clocks": clock_info,
+        "workloads": subs,
         "e2e": e2e,
         "cpu_baseline": cpu,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    pat.close()
     return 0
 
 
@@ -429,102 +568,131 @@ def measure_cfg_largest(pa, dev, hbm, reps: int = 20):
             "shape": [wl.batch, 16, 512, 512], "outputs": "fp32+bf16", "l2": "flushed before each call"}
 
 
-def run_e2e(args, world, local, wl, sets, pat, outs, c_in, u_in, cfg_out, rel, ws, cwl, n_cfg):
-    """Same step, inputs from pinned host memory: per patch, the rows of every layer are
-    copied on a copy stream while the previous patch computes; outputs stream back on a
-    third stream; the guidance inputs go up and the guided eps + rel-MAE come back."""
+def run_e2e(args, world, r: StepRunner):
+    """The same step through the C ABI with its inputs copied from pinned host memory and its
+    outputs copied back, inside the timed region.  Two device input sets and two output sets
+    alternate between steps: step s uploads into set s % 2 on a copy stream (per patch, while
+    the previous patch computes) after the kernels of step s - 2 that read that set are done,
+    and its outputs stream back on a second copy stream before step s + 2 overwrites them.
+    The two host input sets alternate as in the device-resident loop."""
     import patch_attention_b200 as pa
 
-    dev = torch.device("cuda", local)
+    wl, dev = r.wl, r.dev
     B, H, d, N, M, T, L = wl.batch, wl.heads, wl.head_dim, wl.n_img, wl.n_patches, wl.n_txt, wl.n_layers
     P = wl.patch_len
-    host = [{k: v.cpu().pin_memory() for k, v in sets[0][l].items()} for l in range(L)]
-    host_out = [torch.empty(B, N, H, d, dtype=torch.bfloat16).pin_memory() for _ in range(L)]
-    hc, hu = c_in.cpu().pin_memory(), u_in.cpu().pin_memory()
-    hcfg = torch.empty(cfg_out.shape, dtype=torch.bfloat16).pin_memory()
-    hrel = torch.empty(B, dtype=torch.float32).pin_memory()
-    dev_in = [{k: torch.empty_like(v, device=dev) for k, v in host[l].items()} for l in range(L)]
-    dc, du = torch.empty_like(c_in), torch.empty_like(u_in)
+    host = [[{k: v.cpu().pin_memory() for k, v in r.sets[hs][l].items()} for l in range(L)] for hs in range(2)]
+    host_out = [[torch.empty(B, N, H, d, dtype=torch.bfloat16).pin_memory() for _ in range(L)] for _ in range(2)]
+    hc, hu = r.c_in.cpu().pin_memory(), r.u_in.cpu().pin_memory()
+    hcfg = [torch.empty(r.cfg_out.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    hrel = [torch.empty(B, dtype=torch.float32).pin_memory() for _ in range(2)]
+    dev_in = [[{k: torch.empty_like(v, device=dev) for k, v in host[0][l].items()} for l in range(L)] for _ in range(2)]
+    dev_out = [[torch.empty(B, N, H, d, dtype=torch.bfloat16, device=dev) for _ in range(L)] for _ in range(2)]
+    dcu = [(torch.empty_like(r.c_in), torch.empty_like(r.u_in)) for _ in range(2)]
+    dcfg = [torch.empty_like(r.cfg_out) for _ in range(2)]
+    drel = [torch.empty(B, dtype=torch.float32, device=dev) for _ in range(2)]
     comp = torch.cuda.current_stream(dev)
     up = torch.cuda.Stream(dev)
     down = torch.cuda.Stream(dev)
-    ev_in = [torch.cuda.Event() for _ in range(M)]
-    ev_out = [torch.cuda.Event() for _ in range(M)]
-    ev_txt = torch.cuda.Event()
-    ev_cfg = torch.cuda.Event()
+    ev_in = [[torch.cuda.Event() for _ in range(M)] for _ in range(2)]
+    ev_out = [[torch.cuda.Event() for _ in range(M)] for _ in range(2)]
+    ev_txt = [torch.cuda.Event() for _ in range(2)]
+    ev_cfg_in = [torch.cuda.Event() for _ in range(2)]
+    ev_cfg = [torch.cuda.Event() for _ in range(2)]
+    ev_read_done = [None, None]   # compute finished reading dev_in[b] / dcu[b]
+    ev_down_done = [None, None]   # outputs of dev_out[b] / dcfg[b] copied back
     Lb = pa._lib()
     row_bytes = H * d * 2
-    h2d = 0
-    d2h = 0
+    counts = {"h2d": 0, "d2h": 0}
 
-    def one_step():
-        nonlocal h2d, d2h
+    def one_step(s):
+        b = s % 2
+        hs = host[s % 2]
         h2d = d2h = 0
         with torch.cuda.stream(up):
+            if ev_read_done[b] is not None:
+                up.wait_event(ev_read_done[b])  # step s-2's kernels no longer read set b
             for l in range(L):
                 for k in ("k_txt", "v_txt"):
-                    dev_in[l][k].copy_(host[l][k], non_blocking=True)
-                    h2d += host[l][k].numel() * 2
-            ev_txt.record(up)
+                    dev_in[b][l][k].copy_(hs[l][k], non_blocking=True)
+                    h2d += hs[l][k].numel() * 2
+            ev_txt[b].record(up)
             for p in range(M):
                 sl = slice(p * P, (p + 1) * P)
                 for l in range(L):
                     for k in ("q", "k", "v"):
-                        dev_in[l][k][:, sl].copy_(host[l][k][:, sl], non_blocking=True)
-                        h2d += host[l][k][:, sl].numel() * 2
-                ev_in[p].record(up)
-            dc.copy_(hc, non_blocking=True)
-            du.copy_(hu, non_blocking=True)
+                        dev_in[b][l][k][:, sl].copy_(hs[l][k][:, sl], non_blocking=True)
+                        h2d += hs[l][k][:, sl].numel() * 2
+                ev_in[b][p].record(up)
+            dcu[b][0].copy_(hc, non_blocking=True)
+            dcu[b][1].copy_(hu, non_blocking=True)
             h2d += (hc.numel() + hu.numel()) * 4
-        comp.wait_event(ev_txt)
+            ev_cfg_in[b].record(up)
+        if ev_down_done[b] is not None:
+            comp.wait_event(ev_down_done[b])  # step s-2's outputs have been copied back
+        comp.wait_event(ev_txt[b])
         for p in range(M):
-            comp.wait_event(ev_in[p])
+            comp.wait_event(ev_in[b][p])
             off = p * P * row_bytes
             for l in range(L):
-                t = dev_in[l]
-                st = Lb.pf_patch_attn_step(pat.ctx, l, p, t["q"].data_ptr() + off, t["k"].data_ptr() + off,
+                t = dev_in[b][l]
+                st = Lb.pf_patch_attn_step(r.pat.ctx, l, p, t["q"].data_ptr() + off, t["k"].data_ptr() + off,
                                            t["v"].data_ptr() + off, t["k_txt"].data_ptr() if T else None,
-                                           t["v_txt"].data_ptr() if T else None, outs[l].data_ptr() + off,
+                                           t["v_txt"].data_ptr() if T else None, dev_out[b][l].data_ptr() + off,
                                            comp.cuda_stream)
                 if st != 0:
                     raise pa.PatchAttnError(st, "pf_patch_attn_step")
-            ev_out[p].record(comp)
-        comp.wait_stream(up)
-        st = Lb.pf_cfg_combine_relmae(dc.data_ptr(), du.data_ptr(), B, n_cfg, cwl.w, None, cfg_out.data_ptr(),
-                                      rel.data_ptr(), ws.data_ptr(), ws.numel(), comp.cuda_stream)
+            ev_out[b][p].record(comp)
+        comp.wait_event(ev_cfg_in[b])
+        st = Lb.pf_cfg_combine_relmae(dcu[b][0].data_ptr(), dcu[b][1].data_ptr(), B, r.n_cfg, r.cwl.w, None,
+                                      dcfg[b].data_ptr(), drel[b].data_ptr(), r.cws.data_ptr(), r.cws.numel(),
+                                      comp.cuda_stream)
         if st != 0:
             raise pa.PatchAttnError(st, "pf_cfg_combine_relmae")
-        ev_cfg.record(comp)
+        ev_cfg[b].record(comp)
+        e = torch.cuda.Event()
+        e.record(comp)
+        ev_read_done[b] = e
         with torch.cuda.stream(down):
             for p in range(M):
-                down.wait_event(ev_out[p])
+                down.wait_event(ev_out[b][p])
                 sl = slice(p * P, (p + 1) * P)
                 for l in range(L):
-                    host_out[l][:, sl].copy_(outs[l][:, sl], non_blocking=True)
-                    d2h += outs[l][:, sl].numel() * 2
-            down.wait_event(ev_cfg)
-            hcfg.copy_(cfg_out, non_blocking=True)
-            hrel.copy_(rel, non_blocking=True)
-            d2h += cfg_out.numel() * 2 + rel.numel() * 4
-        comp.wait_stream(down)
+                    host_out[b][l][:, sl].copy_(dev_out[b][l][:, sl], non_blocking=True)
+                    d2h += dev_out[b][l][:, sl].numel() * 2
+            down.wait_event(ev_cfg[b])
+            hcfg[b].copy_(dcfg[b], non_blocking=True)
+            hrel[b].copy_(drel[b], non_blocking=True)
+            d2h += dcfg[b].numel() * 2 + drel[b].numel() * 4
+            e2 = torch.cuda.Event()
+            e2.record(down)
+            ev_down_done[b] = e2
+        counts["h2d"], counts["d2h"] = h2d, d2h
 
-    for _ in range(max(1, args.warmup)):
-        one_step()
+    for s in range(max(1, args.warmup)):
+        one_step(s)
     torch.cuda.synchronize(dev)
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize(dev)
     start.record(comp)
-    for _ in range(args.steps):
-        one_step()
+    up.wait_event(start)
+    down.wait_event(start)
+    s0 = max(1, args.warmup)
+    for s in range(s0, s0 + args.steps):
+        one_step(s)
+    comp.wait_stream(up)
+    comp.wait_stream(down)
     stop.record(comp)
     torch.cuda.synchronize(dev)
     barrier(world)
-    pat.check()
+    r.pat.check()
     ms = max_over_ranks(start.elapsed_time(stop) / args.steps, world)
     value = world * L * wl.flop_per_layer_step() / (ms * 1e-3) / 1e12
-    return {"value": value, "unit": "TFLOP/s", "ms_per_step": ms, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "copies": "pinned host, overlapped per patch on two copy streams"}
+    return {"value": value, "unit": "TFLOP/s", "ms_per_step": ms, "h2d_bytes_per_step": counts["h2d"],
+            "d2h_bytes_per_step": counts["d2h"],
+            "copies": "pinned host, two alternating host and device sets, uploads per patch on one "
+                      "copy stream and downloads on another, each buffer reused only after the "
+                      "kernels and copies of the step two before have finished with it"}
 
 
 def run_profile_calls(args):
@@ -575,6 +743,8 @@ def main():
     ap.add_argument("--seed", type=int, default=None)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sub", action="store_true",
+                    help="skip the sd3/pixart sub-records (timed over >= 2 s each)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl != "reference":
         args.warmup = 3

@@ -50,7 +50,9 @@ typedef enum {
   PF_ERR_INVALID_ARG = 1, /* NULL where a pointer is required, negative size, bad layer/patch */
   PF_ERR_SHAPE = 2,       /* n_img not a multiple of n_patches, zero-sized dimension */
   PF_ERR_ALIGN = 3,       /* a device pointer is not 16-byte aligned */
-  PF_ERR_UNSUPPORTED = 4, /* head_dim not in {64, 72, 128}, unknown schedule, no sm_100 device */
+  PF_ERR_UNSUPPORTED = 4, /* head_dim not in {64, 72, 128}, unknown schedule, a current device
+                             that is not compute capability 10.0 (pf_create), or a kernel image
+                             whose compiled register count does not fit its register split */
   PF_ERR_ORDER = 5,       /* patch called out of order for the layer's schedule */
   PF_ERR_STATE = 6,       /* step before pf_kvbuf_init of that layer */
   PF_ERR_CUDA = 7,        /* a CUDA runtime/driver call or a kernel launch failed */
@@ -89,7 +91,10 @@ size_t pf_kvbuf_bytes(const pf_config* cfg);
 
 /* Create a context.  kvbuf_per_layer: host array of n_layers device pointers, each to a
  * caller-owned buffer of pf_kvbuf_bytes(cfg) bytes that must outlive the context.
- * On success *out receives the context; on failure *out is set to NULL. */
+ * On success *out receives the context; on failure *out is set to NULL.
+ * If a CUDA device is current and it is not of compute capability 10.0 (the kernels are
+ * built for sm_100a only), returns PF_ERR_UNSUPPORTED.  With no usable device at all the
+ * context is still created (it is host state only) and its launches return PF_ERR_CUDA. */
 pf_status pf_create(const pf_config* cfg, void* const* kvbuf_per_layer, pf_ctx** out);
 
 /* Free the host state of ctx (not the caller's buffers).  NULL => PF_OK. */
@@ -182,9 +187,9 @@ pf_status pf_cfg_combine_relmae(const float* eps_c, const float* eps_u, int batc
 
 /* Same computation and outputs as pf_cfg_combine_relmae, for callers that cannot allocate
  * device memory: code that runs where another framework owns the device allocator and must
- * see every allocation, loops that cannot afford the device synchronisation a cudaMalloc may
- * imply, or host callbacks that may not make allocation calls.  The pages have no
- * counterpart of this entry point; it is a deployment convenience.
+ * see every allocation, or loops that cannot afford the device synchronisation a cudaMalloc
+ * may imply.  The pages have no counterpart of this entry point; it is a deployment
+ * convenience.
  *
  * The partial sums go to a fixed 64 KiB array inside the library's device image (4096
  * partial-sum pairs) instead of a caller workspace, so the call allocates nothing and takes
@@ -234,9 +239,12 @@ pf_status pf_switch_init(pf_switch* s, float enter_below, int enter_patience, fl
  * the next step.  NaN rel-MAE_t is rejected with PF_ERR_INVALID_ARG and leaves the state. */
 pf_status pf_switch_update(pf_switch* s, float relmae, int* phase_out);
 
-/* Synchronise `stream`, then read the device status word the context's kernels write when
- * a bounded wait expires: PF_ERR_TIMEOUT if any did (and clear it), PF_ERR_CUDA if the
- * stream reported an error, else PF_OK. */
+/* Synchronise `stream`, then read the device status word the kernels write when a bounded
+ * wait expires: PF_ERR_TIMEOUT if any did (and clear it), PF_ERR_CUDA if the stream reported
+ * an error, else PF_OK.  The status word is one per device and process, shared by every
+ * context and stream of the process on that device (the context argument only guards
+ * against NULL): a timeout in any of them is reported, and cleared, by whichever call reads
+ * the word first. */
 pf_status pf_check_device_status(pf_ctx* ctx, void* stream);
 
 /* Self-test of failure detection (the pages have no counterpart): launches a one-thread

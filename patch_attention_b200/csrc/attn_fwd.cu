@@ -42,6 +42,8 @@
 
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "pf_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -56,7 +58,9 @@ __device__ unsigned int g_watchdog = 0;
 // registers, 6 softmax has the row maximum, 7 softmax has P packed, 8 P stored to TMEM.
 constexpr int kTraceTiles = 512;
 // 9 MMA issuer sees the V tile of j-1, 10 producer issued the K (t=0) / V (t=1) tile j.
-__device__ unsigned long long g_trace[11 * 2 * kTraceTiles];
+// The second index is the softmax chain: the query tile (full-row kernels) or 2 * query tile
+// + key half (half-row kernel).
+__device__ unsigned long long g_trace[11 * 4 * kTraceTiles];
 // Per CTA of the latest launch: SM id, start and end (global timer, ns).
 constexpr int kTraceCtas = 4096;
 __device__ unsigned long long g_cta[3 * kTraceCtas];
@@ -71,7 +75,7 @@ __device__ unsigned long long g_cta[3 * kTraceCtas];
   } while (0)
 #define PF_TRACE_AT(ev, t, j)                                                              \
   do {                                                                                     \
-    if (blockIdx.x == 0 && (j) < kTraceTiles) g_trace[((ev) * 2 + (t)) * kTraceTiles + (j)] = clock64(); \
+    if (blockIdx.x == 0 && (j) < kTraceTiles) g_trace[((ev) * 4 + (t)) * kTraceTiles + (j)] = clock64(); \
   } while (0)
 #else
 #define PF_TRACE_AT(ev, t, j) \
@@ -89,13 +93,18 @@ using namespace ptx;
 constexpr int kRows = 128;             // query rows per Q tile == key rows per K/V tile
 constexpr int kChunkBytes = 128 * 128; // 128 rows x 64 bf16 columns (one 128-byte swizzle span)
 constexpr int kThreads = 384;          // 3 warpgroups: softmax 0, softmax 1, MMA/TMA/scatter
-// Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512), the third
-// warpgroup drops to 88 and the two softmax warpgroups rise to 208:
-// 128 x 88 + 256 x 208 = 64512, exactly the registers the CTA was launched with.  (88 keeps
-// the MMA issuer free of spills; 56/224 measured slower.)
+// Register split (setmaxnreg): __launch_bounds__(kThreads, 1) lets the compiler use up to
+// kLaunchRegs = 168 per thread (384 x 168 = 64512 of the SM's 65536), the third warpgroup
+// drops to 88 and the two softmax warpgroups rise to 208: 128 x 88 + 256 x 208 = 64512,
+// exactly the registers the CTA is launched with.  (88 keeps the MMA issuer free of spills;
+// 56/224 measured slower.)  setmaxnreg.inc waits until the CTA's pool can give the registers,
+// so a kernel compiled to fewer registers than the split assumes would wait forever: the
+// host reads the compiled count before the first launch on each device and refuses to launch
+// when the split does not fit (launch_one).
+constexpr int kLaunchRegs = (65536 / kThreads) / 8 * 8;
 constexpr uint32_t kRegsSoftmax = 208;
 constexpr uint32_t kRegsOther = 88;
-static_assert(128 * kRegsOther + 256 * kRegsSoftmax <= kThreads * 168, "register split");
+static_assert(128 * kRegsOther + 256 * kRegsSoftmax <= kThreads * kLaunchRegs, "register split");
 constexpr int kWarpMma = 8;     // TMEM allocation; MMA issuer (of query tile 0 when split)
 constexpr int kWarpMma2 = 11;   // MMA issuer of query tile 1 on the separate-P layout
 constexpr int kWarpLoad = 9;
@@ -137,7 +146,10 @@ struct Segments {
     n_txt = (txt_len + kRows - 1) / kRows;
   }
   __device__ int total() const { return n_fresh + n_lo + n_hi + n_txt; }
-  // src: 0 = fresh tensors, 1 = buffer, 2 = text
+  // src: 0 = fresh tensors, 1 = buffer rows [0, lo_len) through the maps bounded at lo_len
+  // (a ragged last tile reads zeros past the segment, never the rows of patch p that the
+  // scatter of this launch is writing), 2 = text, 3 = buffer rows from hi_row0 (bounded by
+  // the end of the buffer)
   __device__ void tile(int j, int& src, int& row0, int& nvalid) const {
     if (j < n_fresh) {
       src = 0; row0 = j * kRows; nvalid = min(kRows, plen - row0); return;
@@ -148,7 +160,7 @@ struct Segments {
     }
     j -= n_lo;
     if (j < n_hi) {
-      src = 1; row0 = hi_row0 + j * kRows; nvalid = min(kRows, hi_len - j * kRows); return;
+      src = 3; row0 = hi_row0 + j * kRows; nvalid = min(kRows, hi_len - j * kRows); return;
     }
     j -= n_hi;
     src = 2; row0 = j * kRows; nvalid = min(kRows, txt_len - row0);
@@ -310,6 +322,46 @@ __device__ __forceinline__ void raise_abort(volatile int* abort, unsigned code) 
   atomicOr(&g_watchdog, code);
 }
 
+// The scatter warp's work: this CTA's contiguous 1/gridDim share of the flattened
+// [B, P, H, d] fresh K and V, copied into the buffer rows of the patch (16-byte vectors,
+// two in flight per lane).  Nothing when the call has no scatter (k_dst == nullptr).
+template <int D>
+__device__ __forceinline__ void scatter_share(const AttnParams& p, int lane) {
+  if (p.k_dst == nullptr) return;
+  const long long per_b = static_cast<long long>(p.plen) * p.heads * D / 8;  // 16-byte vectors
+  const long long total = per_b * p.batch;
+  const long long lo = total * blockIdx.x / gridDim.x;
+  const long long hi = total * (blockIdx.x + 1) / gridDim.x;
+  const long long img_b = static_cast<long long>(p.n_img) * p.heads * D / 8;
+  const long long patch_off = static_cast<long long>(p.patch) * per_b;
+  const uint4* ksrc = reinterpret_cast<const uint4*>(p.k_p);
+  const uint4* vsrc = reinterpret_cast<const uint4*>(p.v_p);
+  uint4* kdst = reinterpret_cast<uint4*>(p.k_dst);
+  uint4* vdst = reinterpret_cast<uint4*>(p.v_dst);
+  // walk the share one batch element at a time: within one, the destination is the source
+  // index shifted by a constant
+  for (long long bb = lo / per_b; bb * per_b < hi; ++bb) {
+    const long long b_lo = bb * per_b > lo ? bb * per_b : lo;
+    const long long b_hi = (bb + 1) * per_b < hi ? (bb + 1) * per_b : hi;
+    const long long shift = bb * (img_b - per_b) + patch_off;
+    for (long long base = b_lo + lane; base < b_hi; base += 32 * 2) {
+      const long long i1 = base + 32;
+      const uint4 k0 = __ldg(ksrc + base), v0 = __ldg(vsrc + base);
+      uint4 k1, v1;
+      if (i1 < b_hi) {
+        k1 = __ldg(ksrc + i1);
+        v1 = __ldg(vsrc + i1);
+      }
+      kdst[base + shift] = k0;
+      vdst[base + shift] = v0;
+      if (i1 < b_hi) {
+        kdst[i1 + shift] = k1;
+        vdst[i1 + shift] = v1;
+      }
+    }
+  }
+}
+
 template <int D, int NQ>
 __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_constant__ AttnParams p) {
   using Dm = Dims<D>;
@@ -344,8 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
   PF_TRACE_CTA(1);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int part = blockIdx.x / p.n_pairs;
-  const int pair = blockIdx.x - part * p.n_pairs;
+  // pair-major order: the parts of one query-tile pair run in the same wave, so the partials
+  // they write are merged while still in L2, and a wave's CTAs share few heads' context
+  const int pair = blockIdx.x / p.n_split;
+  const int part = blockIdx.x - pair * p.n_split;
   const int grp = pair % p.n_groups;
   const int h = (pair / p.n_groups) % p.heads;
   const int b = pair / (p.n_groups * p.heads);
@@ -379,8 +433,14 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
       prefetch_tmap(&p.tm_kf);
       prefetch_tmap(&p.tm_vf);
     }
-    prefetch_tmap(&p.tm_kb);
-    prefetch_tmap(&p.tm_vb);
+    if (p.lo_len > 0) {
+      prefetch_tmap(&p.tm_kl);
+      prefetch_tmap(&p.tm_vl);
+    }
+    if (p.hi_len > 0) {
+      prefetch_tmap(&p.tm_kb);
+      prefetch_tmap(&p.tm_vb);
+    }
     if (p.n_txt > 0) {
       prefetch_tmap(&p.tm_kt);
       prefetch_tmap(&p.tm_vt);
@@ -428,7 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
             break;
           }
           const CUtensorMap* m = src == 0 ? (kv ? &p.tm_vf : &p.tm_kf)
-                                 : src == 1 ? (kv ? &p.tm_vb : &p.tm_kb)
+                                 : src == 1 ? (kv ? &p.tm_vl : &p.tm_kl)
+                                 : src == 3 ? (kv ? &p.tm_vb : &p.tm_kb)
                                             : (kv ? &p.tm_vt : &p.tm_kt);
           const uint32_t fb = smem_u32(kv_full + st);
           mbar_arrive_expect_tx(fb, Dm::kTileBytes);
@@ -567,42 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
     }
   } else if (warp == kWarpScatter) {
     // ------------------------------------------------------------ buffer scatter
-    // Each CTA copies a contiguous 1/gridDim share of the flattened [B, P, H, d] fresh
-    // K and V into the buffer rows of the patch.
-    if (p.k_dst != nullptr) {
-      const long long per_b = static_cast<long long>(p.plen) * p.heads * D / 8;  // 16-byte vectors
-      const long long total = per_b * p.batch;
-      const long long lo = total * blockIdx.x / gridDim.x;
-      const long long hi = total * (blockIdx.x + 1) / gridDim.x;
-      const long long img_b = static_cast<long long>(p.n_img) * p.heads * D / 8;
-      const long long patch_off = static_cast<long long>(p.patch) * per_b;
-      const uint4* ksrc = reinterpret_cast<const uint4*>(p.k_p);
-      const uint4* vsrc = reinterpret_cast<const uint4*>(p.v_p);
-      uint4* kdst = reinterpret_cast<uint4*>(p.k_dst);
-      uint4* vdst = reinterpret_cast<uint4*>(p.v_dst);
-      // walk the share one batch element at a time: within one, the destination is the
-      // source index shifted by a constant
-      for (long long bb = lo / per_b; bb * per_b < hi; ++bb) {
-        const long long b_lo = bb * per_b > lo ? bb * per_b : lo;
-        const long long b_hi = (bb + 1) * per_b < hi ? (bb + 1) * per_b : hi;
-        const long long shift = bb * (img_b - per_b) + patch_off;
-        for (long long base = b_lo + lane; base < b_hi; base += 32 * 2) {
-          const long long i1 = base + 32;
-          const uint4 k0 = __ldg(ksrc + base), v0 = __ldg(vsrc + base);
-          uint4 k1, v1;
-          if (i1 < b_hi) {
-            k1 = __ldg(ksrc + i1);
-            v1 = __ldg(vsrc + i1);
-          }
-          kdst[base + shift] = k0;
-          vdst[base + shift] = v0;
-          if (i1 < b_hi) {
-            kdst[i1 + shift] = k1;
-            vdst[i1 + shift] = v1;
-          }
-        }
-      }
-    }
+    scatter_share<D>(p, lane);
   }
   } else if (warp < 4 * NQ) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
@@ -905,18 +931,1033 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_co
   }
 }
 
+// Per-device set-up of one instantiation, done once per device before its first launch
+// there (under a lock, so host threads may launch concurrently): the register check of the
+// setmaxnreg split and the dynamic shared memory attribute, which applies to the current
+// device only.
+template <int D, int NQ>
+cudaError_t configure_once(int dev) {
+  static std::mutex mu;
+  static uint64_t done = 0;  // bit per device ordinal
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  const uint64_t bit = 1ull << dev;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done & bit) return cudaSuccess;
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, patch_attn_kernel<D, NQ>);
+  if (e != cudaSuccess) return e;
+  if (128 * static_cast<long>(kRegsOther) + 256 * static_cast<long>(kRegsSoftmax) >
+      static_cast<long>(kThreads) * fa.numRegs)
+    return cudaErrorNotSupported;  // the split would wait forever in setmaxnreg.inc
+  e = cudaFuncSetAttribute(patch_attn_kernel<D, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem_bytes<D, NQ>());
+  if (e != cudaSuccess) return e;
+  done |= bit;
+  return cudaSuccess;
+}
+
 template <int D, int NQ>
 cudaError_t launch_one(const AttnParams& p, cudaStream_t stream) {
-  constexpr int smem = smem_bytes<D, NQ>();
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(patch_attn_kernel<D, NQ>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = configure_once<D, NQ>(dev);
+  if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.n_split);
-  patch_attn_kernel<D, NQ><<<grid, kThreads, smem, stream>>>(p);
+  patch_attn_kernel<D, NQ><<<grid, kThreads, smem_bytes<D, NQ>(), stream>>>(p);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ head_dim 64: half rows
+//
+// With head_dim 64 a key tile costs the tensor core half of what it costs at 128 while the
+// softmax still exponentiates 128 x 128 scores per query tile, so the exponentials, not the
+// MMAs, bound the loop; with one thread per query row there are only two softmax warps per
+// SM sub-partition to keep the special-function unit busy, and each runs a long dependent
+// chain.  This kernel splits every 128-key tile between two softmax warpgroups per query
+// tile: half 0 owns keys 0..63 of each tile, half 1 keys 64..127.  Each half is an
+// independent online softmax over its own keys, with its own reference maximum m, row sum
+// l and O accumulator in TMEM, so the halves never wait for each other inside the loop;
+// they are combined once per CTA, log-sum-exp style (O = (2^(m_0-M) O_0 + 2^(m_1-M) O_1) /
+// (2^(m_0-M) l_0 + 2^(m_1-M) l_1), M = max(m_0, m_1)).  Four softmax warps per
+// sub-partition instead of two.
+//
+// TMEM, per query tile t (256 columns at 256 t): S_0 | S_1 (64 fp32 columns each) | O_0 | O_1
+// (64 each).  P_h (packed bf16) is written over the first 32 columns of S_h, so QK_h(j+1)
+// is issued after PV_h(j) by the same thread; the tensor pipe completes in order, so
+// S_h(j+1) being complete also means PV_h(j) has read P_h(j) and finished O_h.
+//
+// Warps: 0-15 softmax (warp w: query tile w / 8, half (w / 4) % 2, TMEM lane quarter w % 4),
+// 16 TMEM allocation + MMA issuer of query tile 0, 17 TMA producer, 18 scatter, 19 MMA
+// issuer of query tile 1.
+constexpr int kHrThreads = 640;
+constexpr int kHrLaunchRegs = (65536 / kHrThreads) / 8 * 8;  // 96
+constexpr uint32_t kHrRegsSoftmax = 104;
+constexpr uint32_t kHrRegsOther = 56;
+static_assert(128 * kHrRegsOther + 512 * kHrRegsSoftmax <= kHrThreads * kHrLaunchRegs, "register split");
+constexpr int kHrWarpMma0 = 16;
+constexpr int kHrWarpLoad = 17;
+constexpr int kHrWarpScatter = 18;
+constexpr int kHrWarpMma1 = 19;
+constexpr int kHrStages = 8;
+constexpr int kHrTile = kRows * 64 * 2;  // 16 KB: 128 rows x 64 bf16, one 128-byte swizzle span
+constexpr int kHrPoly = 2;               // of every 8 column pairs, exponentiated on the FMA pipe
+
+template <int NQ>
+constexpr int hr_smem_bytes() {
+  return 1024 + (NQ + kHrStages) * kHrTile + 512;
+}
+
+// Maximum of 64 values: 8 independent chains of three-input maxima, then a tree.
+__device__ __forceinline__ float row_max64(const uint32_t (&s)[64]) {
+  float mv[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mv[k] = __uint_as_float(s[k]);
+#pragma unroll
+  for (int k = 8; k < 56; k += 2)
+    mv[(k >> 1) & 7] = max3(mv[(k >> 1) & 7], __uint_as_float(s[k]), __uint_as_float(s[k + 1]));
+  mv[0] = max3(mv[0], mv[4], __uint_as_float(s[56]));
+  mv[1] = max3(mv[1], mv[5], __uint_as_float(s[57]));
+  mv[2] = max3(mv[2], mv[6], __uint_as_float(s[58]));
+  mv[3] = max3(mv[3], mv[7], __uint_as_float(s[59]));
+  mv[0] = max3(mv[0], __uint_as_float(s[60]), __uint_as_float(s[61]));
+  mv[1] = max3(mv[1], __uint_as_float(s[62]), __uint_as_float(s[63]));
+  return max3(mv[0], mv[1], fmaxf(mv[2], mv[3]));
+}
+
+template <int NQ>
+__global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __grid_constant__ AttnParams p) {
+  constexpr int D = 64;
+  constexpr int S = kHrStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + NQ * kHrTile;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + S * kHrTile);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + S;
+  uint64_t* s_full = kv_empty + S;  // [2 t + h]
+  uint64_t* p_full = s_full + 4;    // [2 t + h]
+  uint64_t* o_full = p_full + 4;    // [2 t + h]
+  uint64_t* mma_done = o_full + 4;  // [issuer]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 2);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  __shared__ float xch_m[2][2][kRows];  // [t][h][row]: each half's m and l for the combine
+  __shared__ float xch_l[2][2][kRows];
+  __shared__ int s_last[2];
+
+  PF_TRACE_CTA(1);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // pair-major order: the parts of one query-tile pair run in the same wave, so the partials
+  // they write are merged while still in L2, and a wave's CTAs share few heads' context
+  const int pair = blockIdx.x / p.n_split;
+  const int part = blockIdx.x - pair * p.n_split;
+  const int grp = pair % p.n_groups;
+  const int hd = (pair / p.n_groups) % p.heads;
+  const int b = pair / (p.n_groups * p.heads);
+  const int q0 = grp * NQ * kRows;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(q_full), 1);
+    for (int st = 0; st < S; ++st) {
+      mbar_init(smem_u32(kv_full + st), 1);
+      mbar_init(smem_u32(kv_empty + st), NQ);  // one commit per MMA issuer (one per query tile)
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(smem_u32(s_full + i), 1);
+      mbar_init(smem_u32(p_full + i), 4);  // one arrival per softmax warp of the half
+      mbar_init(smem_u32(o_full + i), 1);
+    }
+    mbar_init(smem_u32(mma_done), 1);
+    mbar_init(smem_u32(mma_done + 1), 1);
+    *abort = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kHrWarpLoad && lane == 0) {
+    prefetch_tmap(&p.tm_q);
+    if (p.fresh_rows > 0) {
+      prefetch_tmap(&p.tm_kf);
+      prefetch_tmap(&p.tm_vf);
+    }
+    if (p.lo_len > 0) {
+      prefetch_tmap(&p.tm_kl);
+      prefetch_tmap(&p.tm_vl);
+    }
+    if (p.hi_len > 0) {
+      prefetch_tmap(&p.tm_kb);
+      prefetch_tmap(&p.tm_vb);
+    }
+    if (p.n_txt > 0) {
+      prefetch_tmap(&p.tm_kt);
+      prefetch_tmap(&p.tm_vt);
+    }
+  }
+  if (warp == kHrWarpMma0) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  Segments seg;
+  seg.init(p);
+  const int n_all = seg.total();
+  const int j0 = static_cast<int>(static_cast<long long>(part) * n_all / p.n_split);
+  const int j1 = static_cast<int>(static_cast<long long>(part + 1) * n_all / p.n_split);
+  const int n_tiles = j1 - j0;  // this CTA's context tiles: j0 .. j1-1
+
+  if (warp >= 16) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kHrRegsOther));
+    if (warp == kHrWarpLoad) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        const uint32_t qbar = smem_u32(q_full);
+        mbar_arrive_expect_tx(qbar, NQ * kHrTile);
+        for (int t = 0; t < NQ; ++t)
+          tma_load_4d(smem_u32(sQ + t * kHrTile), &p.tm_q, 0, hd, q0 + t * kRows, b, qbar);
+        int issued = 0;
+        bool ok = true;
+        for (int j = 0; j < n_tiles && ok; ++j) {
+          int src, row0, nv;
+          seg.tile(j0 + j, src, row0, nv);
+          for (int kv = 0; kv < 2; ++kv) {
+            const int i = 2 * j + kv;
+            const int st = i % S;
+            if (!mbar_wait(smem_u32(kv_empty + st), ((i / S) & 1) ^ 1, abort, kWaitNs)) {
+              ok = false;
+              break;
+            }
+            const CUtensorMap* m = src == 0 ? (kv ? &p.tm_vf : &p.tm_kf)
+                                   : src == 1 ? (kv ? &p.tm_vl : &p.tm_kl)
+                                   : src == 3 ? (kv ? &p.tm_vb : &p.tm_kb)
+                                              : (kv ? &p.tm_vt : &p.tm_kt);
+            const uint32_t fb = smem_u32(kv_full + st);
+            mbar_arrive_expect_tx(fb, kHrTile);
+            tma_load_4d(smem_u32(sKV + st * kHrTile), m, 0, hd, row0, b, fb);
+            issued = i + 1;
+          }
+        }
+        if (!ok) raise_abort(abort, kWdLoad);
+        // drain: every issued copy must land before the CTA exits
+        mbar_wait(qbar, 0, nullptr, kWaitNs);
+        for (int i = issued > S ? issued - S : 0; i < issued; ++i)
+          mbar_wait(smem_u32(kv_full + (i % S)), (i / S) & 1, nullptr, kWaitNs);
+      }
+    } else if (warp == kHrWarpMma0 || (NQ == 2 && warp == kHrWarpMma1)) {
+      // ------------------------------------------------------------ MMA issuer of query tile t
+      if (lane == 0) {
+        const int t = warp == kHrWarpMma0 ? 0 : 1;
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, 0);  // N = 64 keys, K-major K
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 64, 1);  // N = 64 columns, MN-major V
+        const uint32_t q_lo = ((smem_u32(sQ) + t * kHrTile) >> 4) | desc_lbo_bits(16);
+        const uint32_t k_lo = (smem_u32(sKV) >> 4) | desc_lbo_bits(16);
+        const uint32_t v_lo = (smem_u32(sKV) >> 4) | desc_lbo_bits(kChunkBytes);
+        // S_h = Q_t K[64 h .. 64 h + 63]^T: the half's 64 key rows start 64 * 128 bytes in
+        auto issue_qk = [=](int h, int st) {
+          const uint32_t b0 = k_lo + static_cast<uint32_t>((st * kHrTile + h * 8192) >> 4);
+          const uint32_t d = tmem + t * 256 + h * 64;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(d, smem_desc_lo(q_lo + 2 * kk), smem_desc_lo(b0 + 2 * kk), idesc_qk, kk > 0);
+        };
+        // O_h += P_h V[64 h .. 64 h + 63]: P_h from TMEM (over S_h), 16 keys per MMA
+        auto issue_pv = [=](int h, int st, bool acc) {
+          const uint32_t v0 = v_lo + static_cast<uint32_t>((st * kHrTile + h * 8192) >> 4);
+          const uint32_t d = tmem + t * 256 + 128 + h * 64;
+          const uint32_t a = tmem + t * 256 + h * 64;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(d, a + kk * 8, smem_desc_lo(v0 + static_cast<uint32_t>((kk * 2048) >> 4)), idesc_pv,
+                   acc || kk > 0);
+        };
+
+        bool ok = mbar_wait(smem_u32(q_full), 0, abort, kWaitNs);
+        if (ok && n_tiles > 0) {
+          ok = mbar_wait(smem_u32(kv_full + 0), 0, abort, kWaitNs);  // K(0): load 0, stage 0
+          tc_fence_after();
+          if (ok) {
+            issue_qk(0, 0);
+            mma_commit(smem_u32(s_full + 2 * t));
+            issue_qk(1, 0);
+            mma_commit(smem_u32(s_full + 2 * t + 1));
+            mma_commit(smem_u32(kv_empty + 0));
+          }
+        }
+        for (int j = 0; j < n_tiles && ok; ++j) {
+          const int iV = 2 * j + 1, sV = iV % S;
+          if (!(ok = mbar_wait(smem_u32(kv_full + sV), (iV / S) & 1, abort, kWaitNs))) break;
+          const bool has_next = j + 1 < n_tiles;
+          const int iK = 2 * (j + 1), sK = iK % S;
+          if (has_next && !(ok = mbar_wait(smem_u32(kv_full + sK), (iK / S) & 1, abort, kWaitNs))) break;
+          PF_TRACE_AT(4, 2 * t, j);
+          for (int h = 0; h < 2; ++h) {
+            if (!(ok = mbar_wait(smem_u32(p_full + 2 * t + h), j & 1, abort, kWaitNs))) break;
+            tc_fence_after();
+            PF_TRACE_AT(2, 2 * t + h, j);
+            issue_pv(h, sV, j > 0);
+            if (has_next) {
+              issue_qk(h, sK);
+              mma_commit(smem_u32(s_full + 2 * t + h));
+            } else {
+              mma_commit(smem_u32(o_full + 2 * t + h));
+            }
+            PF_TRACE_AT(3, 2 * t + h, j);
+          }
+          if (!ok) break;
+          mma_commit(smem_u32(kv_empty + sV));
+          if (has_next) mma_commit(smem_u32(kv_empty + sK));
+        }
+        if (!ok) raise_abort(abort, kWdMma);
+        // drain every MMA issued by this thread before TMEM is released
+        mma_commit(smem_u32(mma_done + t));
+        mbar_wait(smem_u32(mma_done + t), 0, nullptr, kWaitNs);
+      }
+    } else if (warp == kHrWarpScatter) {
+      // ------------------------------------------------------------ buffer scatter
+      scatter_share<D>(p, lane);
+    }
+  } else if (warp < 8 * NQ) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHrRegsSoftmax));
+    // ------------------------------------------------------------ softmax of one half + epilogue
+    const int t = warp >> 3;
+    const int hh = (warp >> 2) & 1;
+    const int wq = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 256 + hh * 64;
+    const uint32_t tO = tmem + lane_off + t * 256 + 128 + hh * 64;
+    const float c = p.scale_log2;
+    float m = -INFINITY;  // this half's reference row maximum, in log2 units
+    float l = 0.f;
+    bool ok = true;
+    // local indices of this CTA's ragged context tiles and the valid keys of this half there
+    int rag_j[4], rag_nv[4];
+    {
+      const int ends[4] = {seg.n_fresh, seg.n_fresh + seg.n_lo, seg.n_fresh + seg.n_lo + seg.n_hi,
+                           seg.total()};
+      const int lens[4] = {seg.plen, seg.lo_len, seg.hi_len, seg.txt_len};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int e = ends[k] - 1;
+        const int nv = lens[k] % kRows;
+        rag_nv[k] = min(max(nv - 64 * hh, 0), 64);
+        rag_j[k] = (nv != 0 && e >= j0 && e < j1) ? e - j0 : -1;
+      }
+    }
+    for (int j = 0; j < n_tiles; ++j) {
+      ok = mbar_wait(smem_u32(s_full + 2 * t + hh), j & 1, abort, kWaitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      if (wq == 0 && lane == 0) PF_TRACE_AT(0, 2 * t + hh, j);
+      uint32_t s[64];
+      tmem_ld32(tS + 0, s);
+      tmem_ld32(tS + 32, s + 32);
+      tmem_wait_ld();
+      reg_fence<64>(s);
+      int nv = 64;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (j == rag_j[k]) nv = rag_nv[k];
+      if (nv < 64) {
+#pragma unroll
+        for (int k = 0; k < 64; ++k)
+          if (k >= nv) s[k] = __float_as_uint(-INFINITY);
+      }
+      const float mxs = row_max64(s) * c;
+      if (wq == 0 && lane == 0) PF_TRACE_AT(6, 2 * t + hh, j);
+      const bool grow = mxs > m + 8.f;
+      // warp-collective TMEM accesses: the whole warp rescales when any of its rows grew
+      // (alpha is exactly 1 for the others).  S_h(j) being complete means PV_h(j-1) is too.
+      const bool any_grow = __any_sync(0xffffffffu, grow);
+      const float alpha = grow ? ex2(m - mxs) : 1.f;
+      l *= alpha;
+      m = grow ? mxs : m;
+      if (any_grow && j > 0) {
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 16) {
+          uint32_t o[16];
+          tmem_ld16(tO + c0, o);
+          tmem_wait_ld();
+          reg_fence<16>(o);
+#pragma unroll
+          for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_st16(tO + c0, o);
+        }
+      }
+      // a half-row with no valid key so far (its keys all masked) exponentiates against 0:
+      // masked keys then give 0 (or 2^-125 on the polynomial) instead of NaN
+      const float mref = m == -INFINITY ? 0.f : m;
+      uint32_t pk[32];
+      {
+        const float2 cc = make_float2(c, c), nm = make_float2(-mref, -mref);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), cc, nm);
+          const float2 pe = (k & 7) < kHrPoly ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
+          acc[k & 3] = __fadd2_rn(acc[k & 3], pe);
+          pk[k] = pack_bf16(pe.x, pe.y);
+        }
+        const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+        l += a.x + a.y;
+      }
+      if (wq == 0 && lane == 0) PF_TRACE_AT(7, 2 * t + hh, j);
+      tmem_st32(tS, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(p_full + 2 * t + hh));
+      if (wq == 0 && lane == 0) PF_TRACE_AT(1, 2 * t + hh, j);
+    }
+    if (!ok && lane == 0) raise_abort(abort, kWdSoftmax);
+    {
+      bool ok_o = ok && mbar_wait(smem_u32(o_full + 2 * t + hh), 0, abort, kWaitNs);
+      ok_o = __all_sync(0xffffffffu, ok_o);
+      // both halves of the query tile take the same branch (the combine has barriers)
+      ok_o = named_bar_and(1 + t, 2 * kRows, ok_o);
+      if (!ok_o) {
+        if (ok && lane == 0) raise_abort(abort, kWdEpilogue);
+      } else {
+        tc_fence_after();
+        const int rloc = wq * 32 + lane;
+        const int row = q0 + t * kRows + rloc;
+        const bool in_range = row < p.q_rows;
+        // combine the two halves of the row: this thread produces columns 32 hh .. 32 hh + 31
+        xch_m[t][hh][rloc] = m;
+        xch_l[t][hh][rloc] = l;
+        named_bar_sync(1 + t, 2 * kRows);
+        const float m_o = xch_m[t][hh ^ 1][rloc];
+        const float l_o = xch_l[t][hh ^ 1][rloc];
+        const float mrow = fmaxf(m, m_o);  // finite: half 0 has a valid key in every tile
+        const float w_me = ex2(m - mrow), w_o = ex2(m_o - mrow);
+        const float lrow = w_me * l + w_o * l_o;
+        const float w0 = hh == 0 ? w_me : w_o, w1 = hh == 0 ? w_o : w_me;
+        const uint32_t tO0 = tmem + lane_off + t * 256 + 128 + hh * 32;  // O_0 columns of this thread
+        float o[32];
+#pragma unroll
+        for (int c0 = 0; c0 < 32; c0 += 16) {
+          uint32_t a0[16], a1[16];
+          tmem_ld16(tO0 + c0, a0);
+          tmem_ld16(tO0 + 64 + c0, a1);
+          tmem_wait_ld();
+          reg_fence<16>(a0);
+          reg_fence<16>(a1);
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            o[c0 + k] = w0 * __uint_as_float(a0[k]) + w1 * __uint_as_float(a1[k]);
+        }
+        uint16_t* dst = p.o + ((static_cast<size_t>(b) * p.q_rows + row) * p.heads + hd) * D + 32 * hh;
+        if (p.n_split == 1) {
+          const float inv = 1.f / lrow;
+          if (in_range) {
+#pragma unroll
+            for (int k = 0; k < 32; k += 8) {
+              uint4 w;
+              w.x = pack_bf16(o[k + 0] * inv, o[k + 1] * inv);
+              w.y = pack_bf16(o[k + 2] * inv, o[k + 3] * inv);
+              w.z = pack_bf16(o[k + 4] * inv, o[k + 5] * inv);
+              w.w = pack_bf16(o[k + 6] * inv, o[k + 7] * inv);
+              *reinterpret_cast<uint4*>(dst + k) = w;
+            }
+          }
+        } else {
+          // partial: O row (64 columns, this thread's 32), m, l into this part's slot, column-major
+          const size_t slot_elems = static_cast<size_t>(D + 2) * kRows;
+          float* slot0 = p.ws_part + (static_cast<size_t>(pair) * 2 + t) * p.n_split * slot_elems;
+          float* mine = slot0 + static_cast<size_t>(part) * slot_elems;
+#pragma unroll
+          for (int k = 0; k < 32; ++k) mine[(32 * hh + k) * kRows + rloc] = o[k];
+          if (hh == 0) {
+            mine[D * kRows + rloc] = mrow;
+            mine[(D + 1) * kRows + rloc] = lrow;
+          }
+          __threadfence();
+          named_bar_sync(1 + t, 2 * kRows);
+          if (hh == 0 && rloc == 0) {
+            const unsigned old = atomicAdd(p.ws_cnt + pair * 2 + t, 1u);
+            const int last = old == static_cast<unsigned>(p.n_split - 1);
+            if (last) {
+              __threadfence();
+              p.ws_cnt[pair * 2 + t] = 0u;  // ready for the next launch
+            }
+            s_last[t] = last;
+          }
+          named_bar_sync(1 + t, 2 * kRows);
+          if (s_last[t]) {
+            // merge every part of this query tile: this thread's 32 columns of its row
+            float mref = -INFINITY, lsum = 0.f;
+#pragma unroll 4
+            for (int i = 0; i < p.n_split; ++i)
+              mref = fmaxf(mref, __ldcg(slot0 + i * slot_elems + D * kRows + rloc));
+#pragma unroll 4
+            for (int i = 0; i < p.n_split; ++i) {
+              const float* si = slot0 + i * slot_elems;
+              lsum += ex2(__ldcg(si + D * kRows + rloc) - mref) * __ldcg(si + (D + 1) * kRows + rloc);
+            }
+            const float inv = 1.f / lsum;
+            float acc[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) acc[k] = 0.f;
+            for (int i = 0; i < p.n_split; ++i) {
+              const float* si = slot0 + i * slot_elems + rloc;
+              float v[32];
+#pragma unroll
+              for (int k = 0; k < 32; ++k) v[k] = __ldcg(si + (32 * hh + k) * kRows);
+              const float w = ex2(__ldcg(si + D * kRows) - mref) * inv;
+#pragma unroll
+              for (int k = 0; k < 32; ++k) acc[k] = fmaf(w, v[k], acc[k]);
+            }
+            if (in_range) {
+#pragma unroll
+              for (int k = 0; k < 32; k += 8) {
+                uint4 w;
+                w.x = pack_bf16(acc[k + 0], acc[k + 1]);
+                w.y = pack_bf16(acc[k + 2], acc[k + 3]);
+                w.z = pack_bf16(acc[k + 4], acc[k + 5]);
+                w.w = pack_bf16(acc[k + 6], acc[k + 7]);
+                *reinterpret_cast<uint4*>(dst + k) = w;
+              }
+            }
+          }
+        }
+      }
+    }
+  } else {
+    // softmax warps of a second query tile when the CTA has one: idle
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kHrRegsOther));
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  PF_TRACE_CTA(2);
+  if (warp == kHrWarpMma0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int NQ>
+cudaError_t hr_configure_once(int dev) {
+  static std::mutex mu;
+  static uint64_t done = 0;  // bit per device ordinal
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  const uint64_t bit = 1ull << dev;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done & bit) return cudaSuccess;
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, patch_attn_hr_kernel<NQ>);
+  if (e != cudaSuccess) return e;
+  if (128 * static_cast<long>(kHrRegsOther) + 512 * static_cast<long>(kHrRegsSoftmax) >
+      static_cast<long>(kHrThreads) * fa.numRegs)
+    return cudaErrorNotSupported;  // the split would wait forever in setmaxnreg.inc
+  e = cudaFuncSetAttribute(patch_attn_hr_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           hr_smem_bytes<NQ>());
+  if (e != cudaSuccess) return e;
+  done |= bit;
+  return cudaSuccess;
+}
+
+template <int NQ>
+cudaError_t launch_hr(const AttnParams& p, cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = hr_configure_once<NQ>(dev);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.n_split);
+  patch_attn_hr_kernel<NQ><<<grid, kHrThreads, hr_smem_bytes<NQ>(), stream>>>(p);
+  return cudaGetLastError();
+}
+
+// Epilogue of a softmax thread that owns a whole query row: O (TMEM columns from tO) over l
+// to the bf16 output when the call has no key-range split; otherwise the unnormalised row
+// with its m and l goes to this part's workspace slot, and the last part of the query tile
+// to finish (an atomic counter decides) merges all parts.  Called by all 128 threads of the
+// query tile's warpgroup (named barrier 1 + t).
+template <int D>
+__device__ __forceinline__ void full_row_epilogue(const AttnParams& p, uint32_t tO, float m, float l,
+                                                  int pair, int part, int t, int q0, int hd, int b,
+                                                  int wq, int lane, int* s_last) {
+  constexpr int kMmaN = Dims<D>::kMmaN;
+  const int rloc = wq * 32 + lane;
+  const int row = q0 + t * kRows + rloc;
+  uint16_t* dst = p.o + ((static_cast<size_t>(b) * p.q_rows + row) * p.heads + hd) * D;
+  const bool in_range = row < p.q_rows;
+  if (p.n_split == 1) {
+    const float inv = 1.f / l;
+#pragma unroll
+    for (int c0 = 0; c0 < kMmaN; c0 += 16) {
+      uint32_t o[16];
+      tmem_ld16(tO + c0, o);
+      tmem_wait_ld();
+      reg_fence<16>(o);
+      store_row16<D>(dst, c0, o, inv, in_range);
+    }
+    return;
+  }
+  // partial: O row (d columns), m, l into this part's slot, column-major
+  const size_t slot_elems = static_cast<size_t>(D + 2) * kRows;
+  float* slot0 = p.ws_part + (static_cast<size_t>(pair) * 2 + t) * p.n_split * slot_elems;
+  float* mine = slot0 + static_cast<size_t>(part) * slot_elems;
+#pragma unroll
+  for (int c0 = 0; c0 < kMmaN; c0 += 16) {
+    uint32_t o[16];
+    tmem_ld16(tO + c0, o);
+    tmem_wait_ld();
+    reg_fence<16>(o);
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      if (c0 + k < D) mine[(c0 + k) * kRows + rloc] = __uint_as_float(o[k]);
+  }
+  mine[D * kRows + rloc] = m;
+  mine[(D + 1) * kRows + rloc] = l;
+  __threadfence();
+  named_bar_sync(1 + t, kRows);
+  if (rloc == 0) {
+    const unsigned old = atomicAdd(p.ws_cnt + pair * 2 + t, 1u);
+    const int last = old == static_cast<unsigned>(p.n_split - 1);
+    if (last) {
+      __threadfence();
+      p.ws_cnt[pair * 2 + t] = 0u;  // ready for the next launch
+    }
+    s_last[t] = last;
+  }
+  named_bar_sync(1 + t, kRows);
+  if (!s_last[t]) return;
+  // Merge every part of this query tile.  Each round trip to L2 fetches a whole 64-column
+  // block of one part's row (or every part's m and l).
+  float mref = -INFINITY, lsum = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < p.n_split; ++i)
+    mref = fmaxf(mref, __ldcg(slot0 + i * slot_elems + D * kRows + rloc));
+#pragma unroll 4
+  for (int i = 0; i < p.n_split; ++i) {
+    const float* si = slot0 + i * slot_elems;
+    lsum += ex2(__ldcg(si + D * kRows + rloc) - mref) * __ldcg(si + (D + 1) * kRows + rloc);
+  }
+  const float inv = 1.f / lsum;
+#pragma unroll
+  for (int cb = 0; cb < D; cb += 64) {
+    constexpr int kBlock = 64;
+    const int nc = D - cb < kBlock ? D - cb : kBlock;  // constant once unrolled
+    float acc[kBlock];
+#pragma unroll
+    for (int k = 0; k < kBlock; ++k) acc[k] = 0.f;
+    for (int i = 0; i < p.n_split; ++i) {
+      const float* si = slot0 + i * slot_elems + rloc;
+      float v[kBlock];
+#pragma unroll
+      for (int k = 0; k < kBlock; ++k)
+        if (k < nc) v[k] = __ldcg(si + (cb + k) * kRows);
+      const float w = ex2(__ldcg(si + D * kRows) - mref) * inv;
+#pragma unroll
+      for (int k = 0; k < kBlock; ++k)
+        if (k < nc) acc[k] = fmaf(w, v[k], acc[k]);
+    }
+    if (in_range) {
+#pragma unroll
+      for (int k = 0; k < kBlock; k += 8) {
+        if (k < nc) {
+          uint4 w0;
+          w0.x = pack_bf16(acc[k + 0], acc[k + 1]);
+          w0.y = pack_bf16(acc[k + 2], acc[k + 3]);
+          w0.z = pack_bf16(acc[k + 4], acc[k + 5]);
+          w0.w = pack_bf16(acc[k + 6], acc[k + 7]);
+          *reinterpret_cast<uint4*>(dst + cb + k) = w0;
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ head_dim 72/128: split key tiles
+//
+// With one thread per query row and P written over S, the next key tile's QK cannot start
+// before PV has read P, and PV cannot start before the softmax has written P: per query
+// tile the softmax, the PV and the next QK run one after another.  This kernel splits every
+// 128-key tile into two 64-key halves, each with its own S columns and its own P over them.
+// The softmax thread still owns a whole row and keeps one reference maximum m, one row sum l
+// and one O accumulator; it exponentiates half 0 of tile j, hands P_0 to the MMA issuer,
+// then exponentiates half 1 while the tensor core runs PV_0(j) and QK_0(j+1).  By the time
+// the thread comes back to half 0 of tile j+1, its scores are usually ready.
+//
+// TMEM, per query tile t: S_0 | S_1 (64 fp32 columns each) at 128 t, O (head_dim padded to
+// 16 columns) at 256 + 128 t.  An O rescale (the row maximum grew by more than 2^8) must not
+// overlap a PV still accumulating into O: S_h(j) complete implies PV_h(j-1) complete (same
+// issuing thread, issued before QK_h(j)), and the rescale also waits for the other half's
+// latest PV through its own barrier.
+//
+// Warps: 0-7 softmax (warp w: query tile w / 4, TMEM lane quarter w % 4), 8 TMEM allocation
+// + MMA issuer of query tile 0, 9 TMA producer, 10 scatter, 11 MMA issuer of query tile 1.
+template <int D, int NQ>
+__global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid_constant__ AttnParams p) {
+  using Dm = Dims<D>;
+  constexpr int S = Dm::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + NQ * Dm::kTileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + S * Dm::kTileBytes);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + S;
+  uint64_t* s_full = kv_empty + S;   // [2 t + h]
+  uint64_t* p_full = s_full + 4;     // [2 t + h]
+  uint64_t* pv_done = p_full + 4;    // [2 t + h]
+  uint64_t* o_full = pv_done + 4;    // [t]
+  uint64_t* mma_done = o_full + 2;   // [issuer]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 2);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  __shared__ int s_last[2];
+
+  PF_TRACE_CTA(1);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // pair-major order: the parts of one query-tile pair run in the same wave, so the partials
+  // they write are merged while still in L2, and a wave's CTAs share few heads' context
+  const int pair = blockIdx.x / p.n_split;
+  const int part = blockIdx.x - pair * p.n_split;
+  const int grp = pair % p.n_groups;
+  const int hd = (pair / p.n_groups) % p.heads;
+  const int b = pair / (p.n_groups * p.heads);
+  const int q0 = grp * NQ * kRows;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(q_full), 1);
+    for (int st = 0; st < S; ++st) {
+      mbar_init(smem_u32(kv_full + st), 1);
+      mbar_init(smem_u32(kv_empty + st), NQ);  // one commit per MMA issuer (one per query tile)
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(smem_u32(s_full + i), 1);
+      mbar_init(smem_u32(p_full + i), 4);  // one arrival per softmax warp
+      mbar_init(smem_u32(pv_done + i), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(smem_u32(o_full + t), 1);
+      mbar_init(smem_u32(mma_done + t), 1);
+    }
+    *abort = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kWarpLoad && lane == 0) {
+    prefetch_tmap(&p.tm_q);
+    if (p.fresh_rows > 0) {
+      prefetch_tmap(&p.tm_kf);
+      prefetch_tmap(&p.tm_vf);
+    }
+    if (p.lo_len > 0) {
+      prefetch_tmap(&p.tm_kl);
+      prefetch_tmap(&p.tm_vl);
+    }
+    if (p.hi_len > 0) {
+      prefetch_tmap(&p.tm_kb);
+      prefetch_tmap(&p.tm_vb);
+    }
+    if (p.n_txt > 0) {
+      prefetch_tmap(&p.tm_kt);
+      prefetch_tmap(&p.tm_vt);
+    }
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  Segments seg;
+  seg.init(p);
+  const int n_all = seg.total();
+  const int j0 = static_cast<int>(static_cast<long long>(part) * n_all / p.n_split);
+  const int j1 = static_cast<int>(static_cast<long long>(part + 1) * n_all / p.n_split);
+  const int n_tiles = j1 - j0;  // this CTA's context tiles: j0 .. j1-1
+
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+    if (warp == kWarpLoad) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        const uint32_t qbar = smem_u32(q_full);
+        mbar_arrive_expect_tx(qbar, NQ * Dm::kTileBytes);
+        for (int t = 0; t < NQ; ++t)
+          for (int c = 0; c < Dm::kChunks; ++c)
+            tma_load_4d(smem_u32(sQ + t * Dm::kTileBytes + c * kChunkBytes), &p.tm_q, c * 64, hd,
+                        q0 + t * kRows, b, qbar);
+        int issued = 0;
+        bool ok = true;
+        for (int j = 0; j < n_tiles && ok; ++j) {
+          int src, row0, nv;
+          seg.tile(j0 + j, src, row0, nv);
+          for (int kv = 0; kv < 2; ++kv) {
+            const int i = 2 * j + kv;
+            const int st = i % S;
+            if (!mbar_wait(smem_u32(kv_empty + st), ((i / S) & 1) ^ 1, abort, kWaitNs)) {
+              ok = false;
+              break;
+            }
+            const CUtensorMap* m = src == 0 ? (kv ? &p.tm_vf : &p.tm_kf)
+                                   : src == 1 ? (kv ? &p.tm_vl : &p.tm_kl)
+                                   : src == 3 ? (kv ? &p.tm_vb : &p.tm_kb)
+                                              : (kv ? &p.tm_vt : &p.tm_kt);
+            const uint32_t fb = smem_u32(kv_full + st);
+            mbar_arrive_expect_tx(fb, Dm::kTileBytes);
+            for (int c = 0; c < Dm::kChunks; ++c)
+              tma_load_4d(smem_u32(sKV + st * Dm::kTileBytes + c * kChunkBytes), m, c * 64, hd, row0,
+                          b, fb);
+            issued = i + 1;
+          }
+        }
+        if (!ok) raise_abort(abort, kWdLoad);
+        // drain: every issued copy must land before the CTA exits
+        mbar_wait(qbar, 0, nullptr, kWaitNs);
+        for (int i = issued > S ? issued - S : 0; i < issued; ++i)
+          mbar_wait(smem_u32(kv_full + (i % S)), (i / S) & 1, nullptr, kWaitNs);
+      }
+    } else if (warp == kWarpMma || (NQ == 2 && warp == kWarpMma2)) {
+      // ------------------------------------------------------------ MMA issuer of query tile t
+      if (lane == 0) {
+        const int t = warp == kWarpMma ? 0 : 1;
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, 0);         // N = 64 keys
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, Dm::kMmaN, 1);  // N = head_dim (padded)
+        const uint32_t q_lo = ((smem_u32(sQ) + t * Dm::kTileBytes) >> 4) | desc_lbo_bits(16);
+        const uint32_t k_lo = (smem_u32(sKV) >> 4) | desc_lbo_bits(16);
+        const uint32_t v_lo = (smem_u32(sKV) >> 4) | desc_lbo_bits(kChunkBytes);
+        // S_h = Q_t K[64 h .. 64 h + 63]^T: the half's key rows start 64 * 128 bytes into each
+        // 64-column chunk of the K tile
+        auto issue_qk = [=](int h, int st) {
+          const uint32_t b0 = k_lo + static_cast<uint32_t>((st * Dm::kTileBytes + h * 8192) >> 4);
+          const uint32_t d = tmem + t * 128 + h * 64;
+#pragma unroll
+          for (int kk = 0; kk < Dm::kMmaN / 16; ++kk) {
+            const uint32_t off = static_cast<uint32_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+            mma_ss(d, smem_desc_lo(q_lo + off), smem_desc_lo(b0 + off), idesc_qk, kk > 0);
+          }
+        };
+        // O += P_h V[64 h .. 64 h + 63]: P_h from TMEM (over S_h), 16 keys per MMA
+        auto issue_pv = [=](int h, int st, bool acc) {
+          const uint32_t v0 = v_lo + static_cast<uint32_t>((st * Dm::kTileBytes + h * 8192) >> 4);
+          const uint32_t d = tmem + kColO + t * 128;
+          const uint32_t a = tmem + t * 128 + h * 64;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(d, a + kk * 8, smem_desc_lo(v0 + static_cast<uint32_t>((kk * 2048) >> 4)), idesc_pv,
+                   acc || kk > 0);
+        };
+
+        bool ok = mbar_wait(smem_u32(q_full), 0, abort, kWaitNs);
+        if (ok && n_tiles > 0) {
+          ok = mbar_wait(smem_u32(kv_full + 0), 0, abort, kWaitNs);  // K(0): load 0, stage 0
+          tc_fence_after();
+          if (ok) {
+            issue_qk(0, 0);
+            mma_commit(smem_u32(s_full + 2 * t));
+            issue_qk(1, 0);
+            mma_commit(smem_u32(s_full + 2 * t + 1));
+            mma_commit(smem_u32(kv_empty + 0));
+          }
+        }
+        for (int j = 0; j < n_tiles && ok; ++j) {
+          const int iV = 2 * j + 1, sV = iV % S;
+          if (!(ok = mbar_wait(smem_u32(kv_full + sV), (iV / S) & 1, abort, kWaitNs))) break;
+          const bool has_next = j + 1 < n_tiles;
+          const int iK = 2 * (j + 1), sK = iK % S;
+          if (has_next && !(ok = mbar_wait(smem_u32(kv_full + sK), (iK / S) & 1, abort, kWaitNs))) break;
+          PF_TRACE_AT(4, 2 * t, j);
+          for (int h = 0; h < 2; ++h) {
+            if (!(ok = mbar_wait(smem_u32(p_full + 2 * t + h), j & 1, abort, kWaitNs))) break;
+            tc_fence_after();
+            PF_TRACE_AT(2, 2 * t + h, j);
+            issue_pv(h, sV, j > 0 || h > 0);
+            mma_commit(smem_u32(pv_done + 2 * t + h));
+            if (has_next) {
+              issue_qk(h, sK);
+              mma_commit(smem_u32(s_full + 2 * t + h));
+            }
+            PF_TRACE_AT(3, 2 * t + h, j);
+          }
+          if (!ok) break;
+          if (!has_next) mma_commit(smem_u32(o_full + t));
+          mma_commit(smem_u32(kv_empty + sV));
+          if (has_next) mma_commit(smem_u32(kv_empty + sK));
+        }
+        if (!ok) raise_abort(abort, kWdMma);
+        // drain every MMA issued by this thread before TMEM is released
+        mma_commit(smem_u32(mma_done + t));
+        mbar_wait(smem_u32(mma_done + t), 0, nullptr, kWaitNs);
+      }
+    } else if (warp == kWarpScatter) {
+      // ------------------------------------------------------------ buffer scatter
+      scatter_share<D>(p, lane);
+    }
+  } else if (warp < 4 * NQ) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    // ------------------------------------------------------------ softmax + epilogue
+    const int t = warp >> 2;
+    const int wq = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + kColO + t * 128;
+    const float c = p.scale_log2;
+    float m = -INFINITY;  // reference row maximum, in log2 units
+    float l = 0.f;
+    bool ok = true;
+    // local indices of this CTA's ragged context tiles and their valid rows
+    int rag_j[4], rag_nv[4];
+    {
+      const int ends[4] = {seg.n_fresh, seg.n_fresh + seg.n_lo, seg.n_fresh + seg.n_lo + seg.n_hi,
+                           seg.total()};
+      const int lens[4] = {seg.plen, seg.lo_len, seg.hi_len, seg.txt_len};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int e = ends[k] - 1;
+        rag_nv[k] = lens[k] % kRows;
+        rag_j[k] = (rag_nv[k] != 0 && e >= j0 && e < j1) ? e - j0 : -1;
+      }
+    }
+    for (int j = 0; j < n_tiles && ok; ++j) {
+      int nv = kRows;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (j == rag_j[k]) nv = rag_nv[k];
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        ok = mbar_wait(smem_u32(s_full + 2 * t + h), j & 1, abort, kWaitNs);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        if (wq == 0 && lane == 0) PF_TRACE_AT(0, 2 * t + h, j);
+        uint32_t s[64];
+        tmem_ld32(tS + h * 64, s);
+        tmem_ld32(tS + h * 64 + 32, s + 32);
+        tmem_wait_ld();
+        reg_fence<64>(s);
+        const int nvh = min(max(nv - 64 * h, 0), 64);
+        if (nvh < 64) {
+#pragma unroll
+          for (int k = 0; k < 64; ++k)
+            if (k >= nvh) s[k] = __float_as_uint(-INFINITY);
+        }
+        const float mxs = row_max64(s) * c;
+        const bool grow = mxs > m + 8.f;
+        // warp-collective TMEM accesses: the whole warp rescales when any of its rows grew
+        // (alpha is exactly 1 for the others)
+        const bool any_grow = __any_sync(0xffffffffu, grow);
+        const float alpha = grow ? ex2(m - mxs) : 1.f;
+        if (any_grow && (j > 0 || h > 0)) {
+          // O holds earlier PVs: PV_h(j-1) is complete (S_h(j) is); wait for the other
+          // half's latest one, PV_1(j-1) before half 0, PV_0(j) before half 1
+          const uint32_t par = h == 0 ? static_cast<uint32_t>((j - 1) & 1) : static_cast<uint32_t>(j & 1);
+          ok = mbar_wait(smem_u32(pv_done + 2 * t + (h ^ 1)), par, abort, kWaitNs);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
+            uint32_t o[16];
+            tmem_ld16(tO + c0, o);
+            tmem_wait_ld();
+            reg_fence<16>(o);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st16(tO + c0, o);
+          }
+        }
+        l *= alpha;
+        m = grow ? mxs : m;
+        const float mref = m == -INFINITY ? 0.f : m;  // no valid key yet: masked keys give 0
+        uint32_t pk[32];
+        {
+          const float2 cc = make_float2(c, c), nm = make_float2(-mref, -mref);
+          float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                           make_float2(0.f, 0.f)};
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), cc, nm);
+            const float2 pe = (k & 7) < kPolyPairs<D> ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
+            acc[k & 3] = __fadd2_rn(acc[k & 3], pe);
+            pk[k] = pack_bf16(pe.x, pe.y);
+          }
+          const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+          l += a.x + a.y;
+        }
+        if (wq == 0 && lane == 0) PF_TRACE_AT(7, 2 * t + h, j);
+        tmem_st32(tS + h * 64, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(p_full + 2 * t + h));
+        if (wq == 0 && lane == 0) PF_TRACE_AT(1, 2 * t + h, j);
+      }
+    }
+    if (!ok && lane == 0) raise_abort(abort, kWdSoftmax);
+    {
+      bool ok_o = ok && mbar_wait(smem_u32(o_full + t), 0, abort, kWaitNs);
+      ok_o = __all_sync(0xffffffffu, ok_o);
+      // the whole warpgroup takes the same branch (the merge path has barriers)
+      ok_o = named_bar_and(1 + t, kRows, ok_o);
+      if (!ok_o) {
+        if (ok && lane == 0) raise_abort(abort, kWdEpilogue);
+      } else {
+        tc_fence_after();
+        full_row_epilogue<D>(p, tO, m, l, pair, part, t, q0, hd, b, wq, lane, s_last);
+      }
+    }
+  } else {
+    // second softmax warpgroup when the CTA has a single query tile: idle
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  PF_TRACE_CTA(2);
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D, int NQ>
+cudaError_t sn_configure_once(int dev) {
+  static std::mutex mu;
+  static uint64_t done = 0;  // bit per device ordinal
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  const uint64_t bit = 1ull << dev;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done & bit) return cudaSuccess;
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, patch_attn_sn_kernel<D, NQ>);
+  if (e != cudaSuccess) return e;
+  if (128 * static_cast<long>(kRegsOther) + 256 * static_cast<long>(kRegsSoftmax) >
+      static_cast<long>(kThreads) * fa.numRegs)
+    return cudaErrorNotSupported;  // the split would wait forever in setmaxnreg.inc
+  e = cudaFuncSetAttribute(patch_attn_sn_kernel<D, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem_bytes<D, NQ>());
+  if (e != cudaSuccess) return e;
+  done |= bit;
+  return cudaSuccess;
+}
+
+template <int D, int NQ>
+cudaError_t launch_sn(const AttnParams& p, cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = sn_configure_once<D, NQ>(dev);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.n_split);
+  patch_attn_sn_kernel<D, NQ><<<grid, kThreads, smem_bytes<D, NQ>(), stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -972,9 +2013,9 @@ cudaError_t launch_zero_u32(unsigned* p, size_t n, cudaStream_t stream) {
 cudaError_t launch_patch_attn(const AttnParams& p, cudaStream_t stream) {
   const bool two = p.q_rows > kRows;
   switch (p.head_dim) {
-    case 64: return two ? launch_one<64, 2>(p, stream) : launch_one<64, 1>(p, stream);
-    case 72: return two ? launch_one<72, 2>(p, stream) : launch_one<72, 1>(p, stream);
-    case 128: return two ? launch_one<128, 2>(p, stream) : launch_one<128, 1>(p, stream);
+    case 64: return two ? launch_hr<2>(p, stream) : launch_hr<1>(p, stream);
+    case 72: return two ? launch_sn<72, 2>(p, stream) : launch_sn<72, 1>(p, stream);
+    case 128: return two ? launch_sn<128, 2>(p, stream) : launch_sn<128, 1>(p, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -38,17 +39,18 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once per process (thread-safe: the first
+// caller does the lookup, concurrent callers wait for it).
 EncodeTiledFn encode_fn() {
+  static std::once_flag once;
   static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  std::call_once(once, [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
       fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+  });
   return fn;
 }
 
@@ -75,14 +77,18 @@ size_t region_elems(const pf_config* c) {
 }
 
 // [batch, rows, heads, d] bf16 -> 4-D tensor map, box = 64 columns x 1 head x 128 rows.
-bool make_map(CUtensorMap* m, const void* base, int batch, int rows, int heads, int d) {
+// The map covers the first `rows` rows of each batch element, whose rows are `batch_rows`
+// apart (batch_rows >= rows; 0 means rows): loads past `rows` read zeros.
+bool make_map(CUtensorMap* m, const void* base, int batch, int rows, int heads, int d,
+              int batch_rows = 0) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  if (batch_rows == 0) batch_rows = rows;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
                               static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(batch)};
   const cuuint64_t row_bytes = static_cast<cuuint64_t>(heads) * d * 2;
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, row_bytes,
-                                 row_bytes * static_cast<cuuint64_t>(rows)};
+                                 row_bytes * static_cast<cuuint64_t>(batch_rows)};
   const cuuint32_t box[4] = {64, 1, 128, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
@@ -91,6 +97,13 @@ bool make_map(CUtensorMap* m, const void* base, int batch, int rows, int heads, 
 }
 
 pf_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PF_OK : PF_ERR_CUDA; }
+
+// Attention launches: cudaErrorNotSupported is the library's own refusal (a kernel image
+// whose compiled register count does not fit its warpgroup register split).
+pf_status from_attn_launch(cudaError_t e) {
+  if (e == cudaSuccess) return PF_OK;
+  return e == cudaErrorNotSupported ? PF_ERR_UNSUPPORTED : PF_ERR_CUDA;
+}
 
 // (batch, head, query-tile group) pairs of a call with q_rows query rows
 int pairs_for(const pf_config& c, int q_rows) {
@@ -176,6 +189,22 @@ uint8_t* region(const pf_ctx* ctx, int layer, int half, int kv) {
 
 }  // namespace
 
+namespace pf {
+cudaError_t device_is_sm100(bool* ok) {
+  int dev = 0, major = 0, minor = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (e != cudaSuccess) {
+    cudaGetLastError();  // clear the failed query from the thread's last-error slot
+    return e;
+  }
+  // sm_100a code (tcgen05, TMA) runs on compute capability 10.0 only
+  *ok = major == 10 && minor == 0;
+  return cudaSuccess;
+}
+}  // namespace pf
+
 extern "C" {
 
 size_t pf_kvbuf_bytes(const pf_config* cfg) {
@@ -194,6 +223,11 @@ pf_status pf_create(const pf_config* cfg, void* const* kvbuf_per_layer, pf_ctx**
     if (!kvbuf_per_layer[l]) return PF_ERR_INVALID_ARG;
     if (!aligned16(kvbuf_per_layer[l])) return PF_ERR_ALIGN;
   }
+  // A device that is current must be a B200-class part (compute capability 10.0): the
+  // kernels are built for sm_100a only.  Without any usable device the context is still
+  // created (it is host state only); its launches then fail with PF_ERR_CUDA.
+  bool sm100 = false;
+  if (pf::device_is_sm100(&sm100) == cudaSuccess && !sm100) return PF_ERR_UNSUPPORTED;
   pf_ctx* ctx = new (std::nothrow) pf_ctx();
   if (!ctx) return PF_ERR_INVALID_ARG;
   ctx->cfg = *cfg;
@@ -259,11 +293,18 @@ pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
   std::memset(&p, 0, sizeof(p));
   const int read = ctx->read_half[layer];
   const int write = pipefusion ? read : 1 - read;
+  const int lo_len = patch * plen;
   if (!make_map(&p.tm_q, q_p, c.batch, plen, c.heads, d) ||
       !make_map(&p.tm_kf, k_p, c.batch, plen, c.heads, d) ||
       !make_map(&p.tm_vf, v_p, c.batch, plen, c.heads, d) ||
       !make_map(&p.tm_kb, region(ctx, layer, read, 0), c.batch, c.n_img, c.heads, d) ||
       !make_map(&p.tm_vb, region(ctx, layer, read, 1), c.batch, c.n_img, c.heads, d))
+    return PF_ERR_CUDA;
+  // the rows before the patch through maps that end at the patch: the last tile of that
+  // segment reads zeros, not the patch's own rows, which this launch's scatter is writing
+  if (lo_len > 0 &&
+      (!make_map(&p.tm_kl, region(ctx, layer, read, 0), c.batch, lo_len, c.heads, d, c.n_img) ||
+       !make_map(&p.tm_vl, region(ctx, layer, read, 1), c.batch, lo_len, c.heads, d, c.n_img)))
     return PF_ERR_CUDA;
   if (c.n_txt > 0 && (!make_map(&p.tm_kt, k_txt, c.batch, c.n_txt, c.heads, d) ||
                       !make_map(&p.tm_vt, v_txt, c.batch, c.n_txt, c.heads, d)))
@@ -277,10 +318,11 @@ pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
   p.patch = patch;
   p.q_rows = plen;
   p.fresh_rows = plen;
-  p.lo_len = patch * plen;
+  p.lo_len = lo_len;
   p.hi_row0 = (patch + 1) * plen;
   p.hi_len = c.n_img - (patch + 1) * plen;
-  if (launch_attention(ctx, p, stream) != cudaSuccess) return PF_ERR_CUDA;
+  const pf_status ls = from_attn_launch(launch_attention(ctx, p, stream));
+  if (ls != PF_OK) return ls;
 
   if (pipefusion) {
     ctx->next_patch[layer] = (patch + 1) % c.n_patches;
@@ -313,8 +355,8 @@ pf_status pf_text_attn_step(pf_ctx* ctx, int layer, const void* q_txt, const voi
   pf::AttnParams p;
   std::memset(&p, 0, sizeof(p));
   if (!make_map(&p.tm_q, q_txt, c.batch, c.n_txt, c.heads, d) ||
-      !make_map(&p.tm_kb, region(ctx, layer, read, 0), c.batch, c.n_img, c.heads, d) ||
-      !make_map(&p.tm_vb, region(ctx, layer, read, 1), c.batch, c.n_img, c.heads, d) ||
+      !make_map(&p.tm_kl, region(ctx, layer, read, 0), c.batch, c.n_img, c.heads, d) ||
+      !make_map(&p.tm_vl, region(ctx, layer, read, 1), c.batch, c.n_img, c.heads, d) ||
       !make_map(&p.tm_kt, k_txt, c.batch, c.n_txt, c.heads, d) ||
       !make_map(&p.tm_vt, v_txt, c.batch, c.n_txt, c.heads, d))
     return PF_ERR_CUDA;
@@ -325,7 +367,8 @@ pf_status pf_text_attn_step(pf_ctx* ctx, int layer, const void* q_txt, const voi
   p.lo_len = c.n_img;   // the whole buffer as it stands
   p.hi_row0 = c.n_img;
   p.hi_len = 0;
-  if (launch_attention(ctx, p, stream) != cudaSuccess) return PF_ERR_CUDA;
+  const pf_status ls = from_attn_launch(launch_attention(ctx, p, stream));
+  if (ls != PF_OK) return ls;
   return PF_OK;
 }
 

@@ -18,6 +18,8 @@ struct AttnParams {
   CUtensorMap tm_vf;  // V_p
   CUtensorMap tm_kb;  // K buffer being read [B, N, H, d]
   CUtensorMap tm_vb;  // V buffer being read
+  CUtensorMap tm_kl;  // the same buffers bounded at lo_len rows [B, lo_len, H, d]: the rows
+  CUtensorMap tm_vl;  //   past the lo segment are zero-filled, never read (unused if lo_len == 0)
   CUtensorMap tm_kt;  // K_txt [B, T, H, d]  (unused when T == 0)
   CUtensorMap tm_vt;  // V_txt
   const uint16_t* k_p;  // scatter source (fresh rows)
@@ -85,7 +87,8 @@ cudaError_t read_and_clear_watchdog(unsigned* value);
 // and sets its bit in the device word above.
 cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream);
 
-// Host check that a device of compute capability 10.x is current.
-bool device_is_sm100();
+// Whether the current CUDA device is of compute capability 10.0 (what sm_100a code needs).  Returns cudaSuccess and
+// sets *ok, or the error of the device query (no device, no driver).
+cudaError_t device_is_sm100(bool* ok);
 
 }  // namespace pf

@@ -121,9 +121,11 @@ def _close(got, ref, *vs):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("d", [64, 72, 128])
+@pytest.mark.parametrize("d", [8, 64, 72, 128, 256])
 @pytest.mark.parametrize("with_gain", [False, True])
 def test_qk_rmsnorm_matches_oracle(d, with_gain):
+    # d = 8 .. 256 covers every lane-segment width of the kernel (1 .. 32 lanes per vector);
+    # 3330 vectors leave a ragged last group for every width
     g = torch.Generator(device="cuda").manual_seed(d)
     x = (torch.randn(2, 333, 5, d, device="cuda", generator=g) * 2.5).bfloat16()
     x0 = f64(x)

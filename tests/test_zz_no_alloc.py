@@ -1,5 +1,5 @@
 """The no-allocation guidance entry point (pf_cfg_combine_relmae_static) against the
-workspace entry point (pf_cfg_combine_relmae), through the C ABI.
+workspace entry point (pf_cfg_combine_relmae) and the fp64 oracle, through the C ABI.
 
 Some callers cannot allocate device memory at the moment they run the guidance step: the
 device allocator belongs to another framework that must account for every allocation, or
@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import patch_attention_b200 as pa
 from patch_attention_b200 import synth
 
@@ -57,6 +58,32 @@ def test_static_entry_matches_workspace_entry_two_calls():
         got = _static(c, u, w)
         torch.cuda.synchronize()
         _compare(got, _reference(c, u, w), c, u, w)
+
+
+def _compare_with_oracle(got, c, u, w):
+    # same bounds as the workspace entry point's oracle tests: fp32 out within one rounding of
+    # c - u and one fused multiply-add, bf16 out within one bf16 ulp, rel-MAE within 1e-5
+    gf, gb, gr = got
+    B = c.shape[0]
+    cn, un = c.double().cpu().numpy(), u.double().cpu().numpy()
+    ref = oracle.cfg_combine(cn, un, w)
+    _, _, rref = oracle.rel_mae(cn.reshape(B, -1), un.reshape(B, -1))
+    bound = 2.0 ** -22 * (np.abs(un) + abs(w) * np.abs(cn - un)) + 1e-30
+    assert np.all(np.abs(gf.double().cpu().numpy() - ref) <= bound)
+    ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 7)
+    assert np.all(np.abs(gb.double().cpu().numpy() - ref) <= ulp * 1.0001)
+    r = gr.double().cpu().numpy()
+    assert np.all(np.abs(r - rref) <= REL_TOL * np.abs(rref) + 1e-30), (r, rref)
+
+
+def test_static_entry_matches_the_oracle_two_calls():
+    # two calls in a row (the second on a smaller batch, over the array the first one left)
+    w = 7.0
+    for B, shape, t in ((3, (4, 128, 128), 10), (1, (16, 64, 64), 45)):
+        c, u = synth.CfgInputs(synth.CfgWorkload("cfg", B, *shape), device="cuda").step_tensors(t)
+        got = _static(c, u, w)
+        torch.cuda.synchronize()
+        _compare_with_oracle(got, c, u, w)
 
 
 def test_static_entry_rejects_batches_beyond_the_array():
