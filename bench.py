@@ -445,13 +445,38 @@ def measure_copy_kernels(pa, r: StepRunner, hbm, reps=5):
     norm_ms = timed(lambda: pa.pf_qk_rmsnorm(x))
     norm_bytes = 2 * x.numel() * 2
     del x
+    # what the separate pass costs one micro-step: Q_p and K_p of one patch normalised before
+    # the attention launch (the text keys are normalised once per step and layer)
+    P = wl.patch_len
+    qp, kp = t["q"][:, :P].clone(), t["k"][:, :P].clone()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def per_call():
+        flush.zero_()  # the patch's Q and K come from HBM, as they would after the projection
+        e0, e1 = ev(), ev()
+        e0.record(stream)
+        pa.pf_qk_rmsnorm(qp)
+        pa.pf_qk_rmsnorm(kp)
+        e1.record(stream)
+        return e0, e1
+
+    ts = []
+    for i in range(reps + 2):
+        e0, e1 = per_call()
+        torch.cuda.synchronize(dev)
+        if i >= 2:
+            ts.append(e0.elapsed_time(e1))
+    call_norm_ms = statistics.median(ts)
+    del qp, kp, flush
     return {
         "kvbuf_init": {"gb_per_s": init_bytes / (init_ms * 1e-3) / 1e9,
                        "frac_hbm": init_bytes / (init_ms * 1e-3) / 1e9 / hbm, "ms": init_ms,
                        "bytes": init_bytes, "what": f"one {wl.name} layer: K and V [1,{wl.n_img},{wl.heads},{wl.head_dim}] bf16 copied into the buffer"},
         "qk_rmsnorm": {"gb_per_s": norm_bytes / (norm_ms * 1e-3) / 1e9,
                        "frac_hbm": norm_bytes / (norm_ms * 1e-3) / 1e9 / hbm, "ms": norm_ms,
-                       "bytes": norm_bytes, "what": f"in place on a full-spatial {wl.name} Q [1,{wl.n_img},{wl.heads},{wl.head_dim}] bf16"},
+                       "bytes": norm_bytes, "what": f"in place on a full-spatial {wl.name} Q [1,{wl.n_img},{wl.heads},{wl.head_dim}] bf16",
+                       "per_micro_step_ms": call_norm_ms,
+                       "per_micro_step_what": f"Q_p and K_p of one patch [1,{P},{wl.heads},{wl.head_dim}], L2 flushed"},
     }
 
 
@@ -523,7 +548,8 @@ def run_gpu(args, world, rank, local):
                         "peak_source": f"{peak_src} hbm_gbs"},
         "kvbuf_init": copies["kvbuf_init"],
         "scatter": scatter_record(wl, traffic),
-        "qk_rmsnorm": copies["qk_rmsnorm"],
+        "qk_rmsnorm": dict(copies["qk_rmsnorm"], share_of_micro_step=copies["qk_rmsnorm"]["per_micro_step_ms"]
+                           / (copies["qk_rmsnorm"]["per_micro_step_ms"] + roof["launch_ms"])),
         "hbm_peak_gbs": hbm,
         "attn_ms_per_step": attn_ms,
         "gpu_launches": (M * L + 2) * args.steps,

@@ -7,18 +7,18 @@
 // ones), and the step's text tokens are appended (joint attention).  The same launch
 // writes K_p/V_p into the buffer rows of patch p for the calls that follow.
 //
-// Design (per CTA = one head of one batch element, NQ x 128 query rows):
-//   warps 0-3 / 4-7  softmax for query tile 0 / 1: one thread owns one query row (one
-//                    TMEM lane), so the row max and row sum need no shuffles.
-//   warp 8           TMEM allocation and a single-thread tcgen05.mma issuer (of both
-//                    query tiles, or of tile 0 on the separate-P layout).
-//   warp 9           TMA producer: Q tiles once, then K/V tiles through a smem ring.
-//   warp 10          scatter of the CTA's share of K_p/V_p into the buffer.
-//   warp 11          separate-P layout only: the MMA issuer of query tile 1.
-// S = Q K^T lands in TMEM (fp32, 128 columns per query tile); P (packed bf16) is written
-// over S's first 64 columns, or, when head_dim is 64, into the free half of O's columns
-// (the separate-P layout, so the next QK overlaps the softmax).  The PV MMA reads P
-// straight from TMEM (A operand in TMEM, V as an MN-major B operand in smem).  O
+// Two kernels, one per head_dim class, share the rest of the design below:
+//   patch_attn_sn_kernel (head_dim 72, 128): one softmax thread per query row; each
+//     128-key tile is handled as two 64-key halves so that the tensor core runs PV and the
+//     next QK of one half while the softmax exponentiates the other;
+//   patch_attn_hr_kernel (head_dim 64): two softmax threads per query row (each half of the
+//     key tile), four softmax warps per SM sub-partition, for the exponential-bound case.
+// A CTA handles one head of one batch element and NQ (1 or 2) tiles of 128 query rows.
+// Warp roles: softmax warps (one TMEM lane quarter each), one single-thread tcgen05.mma
+// issuer per query tile, a TMA producer (Q once, then K/V tiles through a shared-memory
+// ring), and a scatter warp that copies the CTA's share of K_p/V_p into the buffer.
+// S = Q K^T lands in TMEM (fp32); P is written back to TMEM as packed bf16 and the PV MMA
+// reads it from there (A operand in TMEM, V as an MN-major B operand in shared memory); O
 // accumulates in TMEM.
 // The context is walked as segments so that patch p's rows are read from the fresh
 // tensors, never from buffer rows that other CTAs of this launch are writing:
@@ -93,24 +93,24 @@ using namespace ptx;
 constexpr int kRows = 128;             // query rows per Q tile == key rows per K/V tile
 constexpr int kChunkBytes = 128 * 128; // 128 rows x 64 bf16 columns (one 128-byte swizzle span)
 constexpr int kThreads = 384;          // 3 warpgroups: softmax 0, softmax 1, MMA/TMA/scatter
-// Register split (setmaxnreg): __launch_bounds__(kThreads, 1) lets the compiler use up to
-// kLaunchRegs = 168 per thread (384 x 168 = 64512 of the SM's 65536), the third warpgroup
-// drops to 88 and the two softmax warpgroups rise to 208: 128 x 88 + 256 x 208 = 64512,
-// exactly the registers the CTA is launched with.  (88 keeps the MMA issuer free of spills;
-// 56/224 measured slower.)  setmaxnreg.inc waits until the CTA's pool can give the registers,
-// so a kernel compiled to fewer registers than the split assumes would wait forever: the
-// host reads the compiled count before the first launch on each device and refuses to launch
-// when the split does not fit (launch_one).
+// Register split of patch_attn_sn_kernel (setmaxnreg): __launch_bounds__(kThreads, 1) lets
+// the compiler use up to kLaunchRegs = 168 per thread (384 x 168 = 64512 of the SM's 65536),
+// the third warpgroup drops to 88 and the two softmax warpgroups rise to 208:
+// 128 x 88 + 256 x 208 = 64512, exactly the registers the CTA is launched with.
+// setmaxnreg.inc waits until the CTA's pool can give the registers, so a kernel compiled to
+// fewer registers than the split assumes would wait forever: the host reads the compiled
+// count before the first launch on each device and refuses to launch when the split does not
+// fit (sn_configure_once, hr_configure_once).
 constexpr int kLaunchRegs = (65536 / kThreads) / 8 * 8;
 constexpr uint32_t kRegsSoftmax = 208;
 constexpr uint32_t kRegsOther = 88;
 static_assert(128 * kRegsOther + 256 * kRegsSoftmax <= kThreads * kLaunchRegs, "register split");
-constexpr int kWarpMma = 8;     // TMEM allocation; MMA issuer (of query tile 0 when split)
-constexpr int kWarpMma2 = 11;   // MMA issuer of query tile 1 on the separate-P layout
+constexpr int kWarpMma = 8;     // TMEM allocation; MMA issuer of query tile 0
+constexpr int kWarpMma2 = 11;   // MMA issuer of query tile 1
 constexpr int kWarpLoad = 9;
 constexpr int kWarpScatter = 10;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 256;        // O_t at column 256 + 128 t; S_t at column 128 t
+constexpr uint32_t kColO = 256;        // split-tile kernel: O_t at column 256 + 128 t, S_t at 128 t
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kMaxSplit = 16;          // most key-range parts per query tile
 
@@ -230,86 +230,6 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
-// Maximum of 128 values: 8 independent chains of three-input maxima, then a tree.
-__device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) {
-  float mv[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) mv[k] = __uint_as_float(s[k]);
-#pragma unroll
-  for (int k = 8; k < 120; k += 2)
-    mv[(k >> 1) & 7] = max3(mv[(k >> 1) & 7], __uint_as_float(s[k]), __uint_as_float(s[k + 1]));
-  mv[0] = max3(mv[0], mv[4], __uint_as_float(s[120]));
-  mv[1] = max3(mv[1], mv[5], __uint_as_float(s[121]));
-  mv[2] = max3(mv[2], mv[6], __uint_as_float(s[122]));
-  mv[3] = max3(mv[3], mv[7], __uint_as_float(s[123]));
-  mv[0] = max3(mv[0], __uint_as_float(s[124]), __uint_as_float(s[125]));
-  mv[1] = max3(mv[1], __uint_as_float(s[126]), __uint_as_float(s[127]));
-  return max3(mv[0], mv[1], fmaxf(mv[2], mv[3]));
-}
-
-// p_k = 2^(s_k c - m), packed to bf16 pairs; returns the fp32 sum.  POLY of every 8 pairs
-// of columns use the FMA-pipe polynomial, the rest the special-function unit.  With
-// POLY = 0, masked keys (-inf) give exactly 0 (the polynomial clamps, so masked tiles must
-// use POLY = 0).
-template <int POLY = 0>
-__device__ __forceinline__ void exact_exps(const uint32_t (&s)[128], float c, float m,
-                                           uint32_t (&pk)[64], float& lsum) {
-  const float2 cc = make_float2(c, c), nm = make_float2(-m, -m);
-  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                   make_float2(0.f, 0.f)};
-#pragma unroll
-  for (int k = 0; k < 64; ++k) {
-    const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), cc, nm);
-    const float2 p = (k & 7) < POLY ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
-    acc[k & 3] = __fadd2_rn(acc[k & 3], p);
-    pk[k] = pack_bf16(p.x, p.y);
-  }
-  const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-  lsum = a.x + a.y;
-}
-
-// exact_exps over the column pairs [K0, K1) only, accumulating the fp32 sums into acc (the
-// caller adds acc up): lets a caller place other work between two halves of a row.
-template <int POLY, int K0, int K1>
-__device__ __forceinline__ void exps_span(const uint32_t (&s)[128], float2 cc, float2 nm,
-                                          uint32_t (&pk)[64], float2 (&acc)[4]) {
-#pragma unroll
-  for (int k = K0; k < K1; ++k) {
-    const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), cc, nm);
-    const float2 p = (k & 7) < POLY ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
-    acc[k & 3] = __fadd2_rn(acc[k & 3], p);
-    pk[k] = pack_bf16(p.x, p.y);
-  }
-}
-
-// Same as exact_exps against the current reference m, with POLY of every 8 pairs of
-// columns exponentiated on the FMA pipe; returns max_k (s_k c - m) so the caller can
-// check that no p_k exceeded 2^8.
-template <int POLY>
-__device__ __forceinline__ float speculative_exps(const uint32_t (&s)[128], float c, float m,
-                                                  uint32_t (&pk)[64], float& lsum) {
-  const float2 cc = make_float2(c, c), nm = make_float2(-m, -m);
-  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                   make_float2(0.f, 0.f)};
-  float xm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-  for (int k = 0; k < 64; ++k) {
-    const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), cc, nm);
-    xm[k & 3] = max3(xm[k & 3], x.x, x.y);
-    float2 p;
-    if ((k & 7) < POLY) {
-      p = exp2_poly2(x);
-    } else {
-      p = make_float2(ex2(x.x), ex2(x.y));
-    }
-    acc[k & 3] = __fadd2_rn(acc[k & 3], p);
-    pk[k] = pack_bf16(p.x, p.y);
-  }
-  const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-  lsum = a.x + a.y;
-  return fmaxf(fmaxf(xm[0], xm[1]), fmaxf(xm[2], xm[3]));
-}
-
 // Of every 8 pairs of columns, the pairs whose exponentials run on the FMA pipe instead of
 // the special-function unit.  The polynomial costs about 5 issue slots per element against
 // 1 for the unit (16 results/clk/SM); measured over 0..4 of 8, 2 of 8 was fastest for both
@@ -328,6 +248,8 @@ __device__ __forceinline__ void raise_abort(volatile int* abort, unsigned code) 
 template <int D>
 __device__ __forceinline__ void scatter_share(const AttnParams& p, int lane) {
   if (p.k_dst == nullptr) return;
+  // the previous micro-step reads these buffer rows (as stale context): wait for it
+  grid_dep_wait();
   const long long per_b = static_cast<long long>(p.plen) * p.heads * D / 8;  // 16-byte vectors
   const long long total = per_b * p.batch;
   const long long lo = total * blockIdx.x / gridDim.x;
@@ -362,634 +284,30 @@ __device__ __forceinline__ void scatter_share(const AttnParams& p, int lane) {
   }
 }
 
-template <int D, int NQ>
-__global__ void __launch_bounds__(kThreads, 1) patch_attn_kernel(const __grid_constant__ AttnParams p) {
-  using Dm = Dims<D>;
-  constexpr int S = Dm::kStages;
-  // head_dim 64: O_t needs only 64 of its 128 TMEM columns, so P_t lives in the other 64
-  // instead of over S_t, and the next QK need not wait for the current PV.
-  constexpr bool kSepP = Dm::kMmaN <= 64;
-  // MMA issuing threads.  On the separate-P layout each query tile has its own (a
-  // tcgen05.mma holds its issuing thread for about its execution time, so one thread would
-  // make each tile's next QK wait behind the other tile's PV); on the P-over-S layout one
-  // thread issues for both tiles, which keeps the two softmax warpgroups staggered (two
-  // issuers measured slower there: both tiles' MMAs then contend in lockstep).
-  constexpr int kIssuers = kSepP ? NQ : 1;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sKV = smem + NQ * Dm::kTileBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + S * Dm::kTileBytes);
-  uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = kv_full + S;
-  uint64_t* s_full = kv_empty + S;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_full = p_full + 2;
-  uint64_t* mma_done = o_full + 2;   // [issuer]
-  uint64_t* s_free = mma_done + 2;   // separate-P layout: softmax has S in registers
-  uint64_t* pv_done = s_free + 2;    // separate-P layout: PV of a tile has completed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2);
-  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  PF_TRACE_CTA(1);
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  // pair-major order: the parts of one query-tile pair run in the same wave, so the partials
-  // they write are merged while still in L2, and a wave's CTAs share few heads' context
-  const int pair = blockIdx.x / p.n_split;
-  const int part = blockIdx.x - pair * p.n_split;
-  const int grp = pair % p.n_groups;
-  const int h = (pair / p.n_groups) % p.heads;
-  const int b = pair / (p.n_groups * p.heads);
-  const int q0 = grp * NQ * kRows;
-  __shared__ int s_last[2];
-
-  if (threadIdx.x == 0) {
-    mbar_init(smem_u32(q_full), 1);
-    for (int s = 0; s < S; ++s) {
-      mbar_init(smem_u32(kv_full + s), 1);
-      mbar_init(smem_u32(kv_empty + s), kIssuers);  // one commit per MMA issuer
-    }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(smem_u32(s_full + t), 1);
-      mbar_init(smem_u32(p_full + t), 4);  // one arrival per softmax warp
-      mbar_init(smem_u32(o_full + t), 1);
-    }
-    mbar_init(smem_u32(mma_done), 1);
-    mbar_init(smem_u32(mma_done + 1), 1);
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(smem_u32(s_free + t), 4);  // one arrival per softmax warp
-      mbar_init(smem_u32(pv_done + t), 1);
-    }
-    *abort = 0;
-    fence_mbar_init();
-    fence_proxy_async_smem();
-  }
-  if (warp == kWarpLoad && lane == 0) {
-    prefetch_tmap(&p.tm_q);
-    if (p.fresh_rows > 0) {
-      prefetch_tmap(&p.tm_kf);
-      prefetch_tmap(&p.tm_vf);
-    }
-    if (p.lo_len > 0) {
-      prefetch_tmap(&p.tm_kl);
-      prefetch_tmap(&p.tm_vl);
-    }
-    if (p.hi_len > 0) {
-      prefetch_tmap(&p.tm_kb);
-      prefetch_tmap(&p.tm_vb);
-    }
-    if (p.n_txt > 0) {
-      prefetch_tmap(&p.tm_kt);
-      prefetch_tmap(&p.tm_vt);
-    }
-  }
-  if (warp == kWarpMma) {
-    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  Segments seg;
-  seg.init(p);
-  const int n_all = seg.total();
-  const int j0 = static_cast<int>(static_cast<long long>(part) * n_all / p.n_split);
-  const int j1 = static_cast<int>(static_cast<long long>(part + 1) * n_all / p.n_split);
-  const int n_tiles = j1 - j0;  // this CTA's context tiles: j0 .. j1-1
-
-  if (warp >= 8) {
-  // Every warp of a warpgroup executes the same setmaxnreg, inside the branch whose code
-  // runs under that register budget.
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
-  if (warp == kWarpLoad) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      const uint32_t qbar = smem_u32(q_full);
-      mbar_arrive_expect_tx(qbar, NQ * Dm::kTileBytes);
-      for (int t = 0; t < NQ; ++t)
-        for (int c = 0; c < Dm::kChunks; ++c)
-          tma_load_4d(smem_u32(sQ + t * Dm::kTileBytes + c * kChunkBytes), &p.tm_q, c * 64, h,
-                      q0 + t * kRows, b, qbar);
-      int issued = 0;
-      bool ok = true;
-      for (int j = 0; j < n_tiles && ok; ++j) {
-        int src, row0, nv;
-        seg.tile(j0 + j, src, row0, nv);
-        for (int kv = 0; kv < 2; ++kv) {
-          const int i = 2 * j + kv;
-          const int st = i % S;
-          if (!mbar_wait(smem_u32(kv_empty + st), ((i / S) & 1) ^ 1, abort, kWaitNs)) {
-            ok = false;
-            break;
-          }
-          const CUtensorMap* m = src == 0 ? (kv ? &p.tm_vf : &p.tm_kf)
-                                 : src == 1 ? (kv ? &p.tm_vl : &p.tm_kl)
-                                 : src == 3 ? (kv ? &p.tm_vb : &p.tm_kb)
-                                            : (kv ? &p.tm_vt : &p.tm_kt);
-          const uint32_t fb = smem_u32(kv_full + st);
-          mbar_arrive_expect_tx(fb, Dm::kTileBytes);
-          for (int c = 0; c < Dm::kChunks; ++c)
-            tma_load_4d(smem_u32(sKV + st * Dm::kTileBytes + c * kChunkBytes), m, c * 64, h, row0,
-                        b, fb);
-          issued = i + 1;
-          PF_TRACE_AT(10, kv, j);
-        }
-      }
-      if (!ok) raise_abort(abort, kWdLoad);
-      // drain: every issued copy must land before the CTA exits
-      mbar_wait(qbar, 0, nullptr, kWaitNs);
-      for (int i = issued > S ? issued - S : 0; i < issued; ++i)
-        mbar_wait(smem_u32(kv_full + (i % S)), (i / S) & 1, nullptr, kWaitNs);
-    }
-  } else if (warp == kWarpMma || (kIssuers == 2 && warp == kWarpMma2)) {
-    // ------------------------------------------------------------ MMA issuer(s)
-    if (lane == 0) {
-      const int me = warp == kWarpMma ? 0 : 1;  // issuer index (the query tile, when split)
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, Dm::kMmaN, 1);
-      const uint32_t q_base = smem_u32(sQ);
-      const uint32_t kv_base = smem_u32(sKV);
-
-      // Descriptor low words (start address >> 4 | LBO) of the operand bases; an operand at
-      // byte offset `off` from a base only adds off >> 4 to the 14-bit start-address field
-      // (no carry: shared memory < 256 KB).  The high word is a compile-time constant.
-      const uint32_t q_lo = (q_base >> 4) | desc_lbo_bits(16);
-      const uint32_t k_lo = (kv_base >> 4) | desc_lbo_bits(16);
-      const uint32_t v_lo = (kv_base >> 4) | desc_lbo_bits(kChunkBytes);
-      auto issue_qk = [=](int t, int st) {
-        const uint32_t a0 = q_lo + static_cast<uint32_t>((t * Dm::kTileBytes) >> 4);
-        const uint32_t b0 = k_lo + static_cast<uint32_t>((st * Dm::kTileBytes) >> 4);
-        const uint32_t d = tmem + t * 128;
-#pragma unroll
-        for (int kk = 0; kk < Dm::kMmaN / 16; ++kk) {
-          const uint32_t off = static_cast<uint32_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
-          mma_ss(d, smem_desc_lo(a0 + off), smem_desc_lo(b0 + off), idesc_qk, kk > 0);
-        }
-      };
-      auto issue_pv = [=](int t, int st, bool acc) {
-        const uint32_t v0 = v_lo + static_cast<uint32_t>((st * Dm::kTileBytes) >> 4);
-        const uint32_t d = tmem + kColO + t * 128;
-        const uint32_t a = tmem + (kSepP ? kColO + t * 128 + 64 : t * 128);
-#pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk)
-          mma_ts(d, a + kk * 8, smem_desc_lo(v0 + static_cast<uint32_t>((kk * 2048) >> 4)), idesc_pv,
-                 acc || kk > 0);
-      };
-
-      bool ok = mbar_wait(smem_u32(q_full), 0, abort, kWaitNs);
-      tc_fence_after();
-      if constexpr (kSepP) {
-        // P has its own TMEM columns: QK of the next key tile is issued as soon as the
-        // softmax has S of the current one in registers, so the tensor core computes
-        // S(j+1) while the softmax is still exponentiating tile j.
-        const int t = me;  // this issuer's query tile
-        if (ok && n_tiles > 0) {
-          ok = mbar_wait(smem_u32(kv_full + 0), 0, abort, kWaitNs);  // K(0): load 0, stage 0
-          tc_fence_after();
-          if (ok) {
-            issue_qk(t, 0);
-            mma_commit(smem_u32(s_full + t));
-            mma_commit(smem_u32(kv_empty + 0));
-          }
-        }
-        for (int j = 0; j < n_tiles && ok; ++j) {
-          if (j + 1 < n_tiles) {
-            const int iK = 2 * (j + 1), sK = iK % S;
-            if (!(ok = mbar_wait(smem_u32(kv_full + sK), (iK / S) & 1, abort, kWaitNs))) break;
-            if (t == 0) PF_TRACE_AT(4, 0, j + 1);
-            if (!(ok = mbar_wait(smem_u32(s_free + t), j & 1, abort, kWaitNs))) break;
-            tc_fence_after();
-            issue_qk(t, sK);
-            mma_commit(smem_u32(s_full + t));
-            mma_commit(smem_u32(kv_empty + sK));
-            PF_TRACE_AT(3, t, j + 1);
-          }
-          const int iV = 2 * j + 1, sV = iV % S;
-          if (!(ok = mbar_wait(smem_u32(kv_full + sV), (iV / S) & 1, abort, kWaitNs))) break;
-          if (t == 0) PF_TRACE_AT(9, 0, j);
-          if (!(ok = mbar_wait(smem_u32(p_full + t), j & 1, abort, kWaitNs))) break;
-          tc_fence_after();
-          PF_TRACE_AT(2, t, j);
-          issue_pv(t, sV, j > 0);
-          mma_commit(smem_u32(pv_done + t));
-          mma_commit(smem_u32(kv_empty + sV));
-        }
-      } else {
-      for (int j = 0; j < n_tiles && ok; ++j) {
-        const int iK = 2 * j, sK = iK % S;
-        if (!(ok = mbar_wait(smem_u32(kv_full + sK), (iK / S) & 1, abort, kWaitNs))) break;
-        tc_fence_after();
-        PF_TRACE_AT(4, 0, j);
-        int sV = 0;
-        if (j > 0) {
-          const int iV = 2 * j - 1;
-          sV = iV % S;
-          if (!(ok = mbar_wait(smem_u32(kv_full + sV), (iV / S) & 1, abort, kWaitNs))) break;
-          PF_TRACE_AT(9, 0, j - 1);
-          tc_fence_after();
-        }
-        for (int t = 0; t < NQ; ++t) {
-          if (j > 0) {
-            if (!(ok = mbar_wait(smem_u32(p_full + t), (j - 1) & 1, abort, kWaitNs))) break;
-            tc_fence_after();
-            PF_TRACE_AT(2, t, j - 1);
-            issue_pv(t, sV, j - 1 > 0);
-          }
-          issue_qk(t, sK);
-          mma_commit(smem_u32(s_full + t));
-          PF_TRACE_AT(3, t, j);
-        }
-        if (!ok) break;
-        mma_commit(smem_u32(kv_empty + sK));
-        if (j > 0) mma_commit(smem_u32(kv_empty + sV));
-      }
-      if (ok && n_tiles > 0) {
-        const int iV = 2 * n_tiles - 1, sV = iV % S;
-        ok = mbar_wait(smem_u32(kv_full + sV), (iV / S) & 1, abort, kWaitNs);
-        tc_fence_after();
-        for (int t = 0; t < NQ && ok; ++t) {
-          if (!(ok = mbar_wait(smem_u32(p_full + t), (n_tiles - 1) & 1, abort, kWaitNs))) break;
-          tc_fence_after();
-          issue_pv(t, sV, n_tiles - 1 > 0);
-          mma_commit(smem_u32(o_full + t));
-        }
-        if (ok) mma_commit(smem_u32(kv_empty + sV));
-      }
-      }
-      if (!ok) raise_abort(abort, kWdMma);
-      // drain every MMA issued by this thread before TMEM is released
-      mma_commit(smem_u32(mma_done + me));
-      mbar_wait(smem_u32(mma_done + me), 0, nullptr, kWaitNs);
-    }
-  } else if (warp == kWarpScatter) {
-    // ------------------------------------------------------------ buffer scatter
-    scatter_share<D>(p, lane);
-  }
-  } else if (warp < 4 * NQ) {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-    // ------------------------------------------------------------ softmax + epilogue
-    const int t = warp >> 2;
-    const int wq = warp & 3;
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + t * 128;
-    const uint32_t tO = tmem + lane_off + kColO + t * 128;
-    const float c = p.scale_log2;
-    float m = -INFINITY;  // reference row maximum, already scaled to log2 units
-    float l = 0.f;
-    bool ok = true;
-    // Local indices of this CTA's context tiles with fewer than 128 valid rows (the last tile
-    // of a segment whose length is not a multiple of 128; -1 if not in range) and their
-    // valid row counts, so the loop needs no segment arithmetic.
-    int rag_j[4], rag_nv[4];
-    {
-      const int ends[4] = {seg.n_fresh, seg.n_fresh + seg.n_lo, seg.n_fresh + seg.n_lo + seg.n_hi,
-                           seg.total()};
-      const int lens[4] = {seg.plen, seg.lo_len, seg.hi_len, seg.txt_len};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int e = ends[k] - 1;
-        rag_nv[k] = lens[k] % kRows;
-        rag_j[k] = (rag_nv[k] != 0 && e >= j0 && e < j1) ? e - j0 : -1;
-      }
-    }
-    bool s_ready = false;  // separate-P layout: S(j) was seen complete at the end of tile j-1
-    for (int j = 0; j < n_tiles; ++j) {
-      if (!s_ready) {
-        ok = mbar_wait(smem_u32(s_full + t), j & 1, abort, kWaitNs);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-      }
-      tc_fence_after();
-      if (wq == 0 && lane == 0) PF_TRACE_AT(0, t, j);
-      uint32_t s[128];
-      tmem_ld32(tS + 0, s);
-      tmem_ld32(tS + 32, s + 32);
-      tmem_ld32(tS + 64, s + 64);
-      tmem_ld32(tS + 96, s + 96);
-      tmem_wait_ld();
-      reg_fence<128>(s);
-      if (wq == 0 && lane == 0) PF_TRACE_AT(5, t, j);
-      int nv = kRows;
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (j == rag_j[k]) nv = rag_nv[k];
-      uint32_t pk[64];
-      float lsum;
-      if constexpr (kSepP) {
-        // S is in registers: hand its TMEM columns back so QK of the next tile can start.
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(s_free + t));
-        if (nv < kRows) {
-#pragma unroll
-          for (int k = 0; k < 128; ++k)
-            if (k >= nv) s[k] = __float_as_uint(-INFINITY);
-        }
-        // Reference maximum, updated without a branch (the O rescale it may need is done
-        // after the exponentials, before P is published).
-        const float mxs = row_max128(s) * c;
-        if (wq == 0 && lane == 0) PF_TRACE_AT(6, t, j);
-        const bool grow = mxs > m + 8.f;
-        // the O rescale below uses warp-collective TMEM accesses: the whole warp takes it
-        // when any of its rows grew (alpha is exactly 1 for the others)
-        const bool any_grow = __any_sync(0xffffffffu, grow);
-        const float alpha = grow ? ex2(m - mxs) : 1.f;
-        l *= alpha;
-        m = grow ? mxs : m;
-        // P(j) may overwrite P(j-1) only once PV(j-1) has read it.  QK(j+1) was issued by
-        // the same thread after PV(j-1) and the tensor pipe completes in order, so S(j+1)
-        // being complete implies it -- and S(j+1) is what the next tile waits for anyway.
-        // The last tile waits for PV(j-1) itself.  The barrier is probed half way through
-        // the exponentials so that the wait is usually already over.
-        const bool has_next = j + 1 < n_tiles;
-        const uint32_t gate = has_next ? smem_u32(s_full + t) : smem_u32(pv_done + t);
-        const uint32_t gate_par = has_next ? static_cast<uint32_t>((j + 1) & 1)
-                                           : static_cast<uint32_t>((j - 1) & 1);
-        bool gate_ok = !has_next && j == 0;  // a single tile: nothing to wait for
-        // Masked keys (-inf) give exactly 0 on the special-function unit and 2^-125 on the
-        // polynomial, which is below any sum that includes the row maximum's own term (1),
-        // so ragged tiles use the same mix.
-        {
-          const float2 cc = make_float2(c, c), nm = make_float2(-m, -m);
-          float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                           make_float2(0.f, 0.f)};
-          exps_span<kPolyPairs<D>, 0, 32>(s, cc, nm, pk, acc);
-          if (!gate_ok) gate_ok = mbar_test_wait_all(gate, gate_par);
-          exps_span<kPolyPairs<D>, 32, 64>(s, cc, nm, pk, acc);
-          const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-          lsum = a.x + a.y;
-        }
-        l += lsum;
-        if (!gate_ok) {
-          ok = mbar_wait(gate, gate_par, abort, kWaitNs);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-        }
-        tc_fence_after();
-        s_ready = has_next;
-        if (any_grow && j > 0) {
-#pragma unroll
-          for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
-            uint32_t o[16];
-            tmem_ld16(tO + c0, o);
-            tmem_wait_ld();
-            reg_fence<16>(o);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st16(tO + c0, o);
-          }
-        }
-        if (wq == 0 && lane == 0) PF_TRACE_AT(7, t, j);
-        tmem_st32(tO + 64, pk);
-        tmem_st32(tO + 96, pk + 32);
-        tmem_wait_st();
-        if (wq == 0 && lane == 0) PF_TRACE_AT(8, t, j);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(p_full + t));
-        if (wq == 0 && lane == 0) PF_TRACE_AT(1, t, j);
-        continue;
-      }
-      // Fast path: exponentiate against the current reference maximum m straight away and
-      // check afterwards that no value exceeded 2^8; the row maximum is then off the
-      // critical path.  The first tile (no reference yet), ragged tiles (masked keys) and
-      // the rare tile whose maximum grew by more than 2^8 take the exact path instead.
-      bool exact = (j == 0) || (nv < kRows);
-      if (!exact) {
-        float xm = speculative_exps<kPolyPairs<D>>(s, c, m, pk, lsum);
-        // warp-uniform decision (the reload is a warp-collective TMEM access): if any row of
-        // the warp exceeded 2^8, the whole warp redoes the tile exactly
-        if (__any_sync(0xffffffffu, xm > 8.f)) {
-          // S is still in TMEM (P has not been written yet): reload it for the exact path
-          exact = true;
-          tmem_ld32(tS + 0, s);
-          tmem_ld32(tS + 32, s + 32);
-          tmem_ld32(tS + 64, s + 64);
-          tmem_ld32(tS + 96, s + 96);
-          tmem_wait_ld();
-          reg_fence<128>(s);
-        }
-      }
-      if (exact) {
-        if (nv < kRows) {
-#pragma unroll
-          for (int k = 0; k < 128; ++k)
-            if (k >= nv) s[k] = __float_as_uint(-INFINITY);
-        }
-        const float mxs = row_max128(s) * c;
-        const bool grow = mxs > m + 8.f;
-        const float alpha = grow ? ex2(m - mxs) : 1.f;
-        l *= alpha;
-        m = grow ? mxs : m;
-        // warp-collective TMEM accesses: the whole warp rescales when any row grew
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
-#pragma unroll
-          for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
-            uint32_t o[16];
-            tmem_ld16(tO + c0, o);
-            tmem_wait_ld();
-            reg_fence<16>(o);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st16(tO + c0, o);
-          }
-        }
-        exact_exps(s, c, m, pk, lsum);
-      }
-      l += lsum;
-      if (wq == 0 && lane == 0) PF_TRACE_AT(7, t, j);
-      tmem_st32(tS, pk);
-      tmem_st32(tS + 32, pk + 32);
-      tmem_wait_st();
-      if (wq == 0 && lane == 0) PF_TRACE_AT(8, t, j);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(p_full + t));
-      if (wq == 0 && lane == 0) PF_TRACE_AT(1, t, j);
-    }
-    if (!ok && lane == 0) raise_abort(abort, kWdSoftmax);
-    {
-      // final O: the last PV of this tile (separate-P layout) or the o_full commit
-      bool ok_o = ok && (kSepP ? mbar_wait(smem_u32(pv_done + t), (n_tiles - 1) & 1, abort, kWaitNs)
-                               : mbar_wait(smem_u32(o_full + t), 0, abort, kWaitNs));
-      ok_o = __all_sync(0xffffffffu, ok_o);
-      // the whole warpgroup takes the same branch (the merge path has barriers)
-      ok_o = named_bar_and(1 + t, kRows, ok_o);
-      if (!ok_o) {
-        if (ok && lane == 0) raise_abort(abort, kWdEpilogue);
-      } else {
-        tc_fence_after();
-        const int rloc = wq * 32 + lane;
-        const int row = q0 + t * kRows + rloc;
-        uint16_t* dst = p.o + ((static_cast<size_t>(b) * p.q_rows + row) * p.heads + h) * D;
-        const bool in_range = row < p.q_rows;
-        if (p.n_split == 1) {
-          const float inv = 1.f / l;
-#pragma unroll
-          for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
-            uint32_t o[16];
-            tmem_ld16(tO + c0, o);
-            tmem_wait_ld();
-            reg_fence<16>(o);
-            store_row16<D>(dst, c0, o, inv, in_range);
-          }
-        } else {
-          // partial: O row (d columns), m, l into this part's slot, column-major
-          const size_t slot_elems = static_cast<size_t>(D + 2) * kRows;
-          float* slot0 = p.ws_part + (static_cast<size_t>(pair) * 2 + t) * p.n_split * slot_elems;
-          float* mine = slot0 + static_cast<size_t>(part) * slot_elems;
-#pragma unroll
-          for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
-            uint32_t o[16];
-            tmem_ld16(tO + c0, o);
-            tmem_wait_ld();
-            reg_fence<16>(o);
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-              if (c0 + k < D) mine[(c0 + k) * kRows + rloc] = __uint_as_float(o[k]);
-          }
-          mine[D * kRows + rloc] = m;
-          mine[(D + 1) * kRows + rloc] = l;
-          __threadfence();
-          named_bar_sync(1 + t, kRows);
-          if (rloc == 0) {
-            const unsigned old = atomicAdd(p.ws_cnt + pair * 2 + t, 1u);
-            const int last = old == static_cast<unsigned>(p.n_split - 1);
-            if (last) {
-              __threadfence();
-              p.ws_cnt[pair * 2 + t] = 0u;  // ready for the next launch
-            }
-            s_last[t] = last;
-          }
-          named_bar_sync(1 + t, kRows);
-          if (s_last[t]) {
-            // Merge every part of this query tile.  The loads are arranged so that each
-            // round trip to L2 fetches a whole 64-column block of one part's row (or every
-            // part's m and l), instead of one dependent round per 8 columns and part.
-            float mref = -INFINITY, lsum = 0.f;
-#pragma unroll 4
-            for (int i = 0; i < p.n_split; ++i)
-              mref = fmaxf(mref, __ldcg(slot0 + i * slot_elems + D * kRows + rloc));
-#pragma unroll 4
-            for (int i = 0; i < p.n_split; ++i) {
-              const float* si = slot0 + i * slot_elems;
-              lsum += ex2(__ldcg(si + D * kRows + rloc) - mref) * __ldcg(si + (D + 1) * kRows + rloc);
-            }
-            const float inv = 1.f / lsum;
-#pragma unroll
-            for (int cb = 0; cb < D; cb += 64) {
-              constexpr int kBlock = 64;
-              const int nc = D - cb < kBlock ? D - cb : kBlock;  // constant once unrolled
-              float acc[kBlock];
-#pragma unroll
-              for (int k = 0; k < kBlock; ++k) acc[k] = 0.f;
-              for (int i = 0; i < p.n_split; ++i) {
-                const float* si = slot0 + i * slot_elems + rloc;
-                float v[kBlock];
-#pragma unroll
-                for (int k = 0; k < kBlock; ++k)
-                  if (k < nc) v[k] = __ldcg(si + (cb + k) * kRows);
-                const float w = ex2(__ldcg(si + D * kRows) - mref) * inv;
-#pragma unroll
-                for (int k = 0; k < kBlock; ++k)
-                  if (k < nc) acc[k] = fmaf(w, v[k], acc[k]);
-              }
-              if (in_range) {
-#pragma unroll
-                for (int k = 0; k < kBlock; k += 8) {
-                  if (k < nc) {
-                    uint4 w0;
-                    w0.x = pack_bf16(acc[k + 0], acc[k + 1]);
-                    w0.y = pack_bf16(acc[k + 2], acc[k + 3]);
-                    w0.z = pack_bf16(acc[k + 4], acc[k + 5]);
-                    w0.w = pack_bf16(acc[k + 6], acc[k + 7]);
-                    *reinterpret_cast<uint4*>(dst + cb + k) = w0;
-                  }
-                }
-              }
-            }
-          }
-        }
-      }
-    }
-  } else {
-    // second softmax warpgroup when the CTA has a single query tile: idle
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  PF_TRACE_CTA(2);
-  if (warp == kWarpMma) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
-  }
-}
-
-// Per-device set-up of one instantiation, done once per device before its first launch
-// there (under a lock, so host threads may launch concurrently): the register check of the
-// setmaxnreg split and the dynamic shared memory attribute, which applies to the current
-// device only.
-template <int D, int NQ>
-cudaError_t configure_once(int dev) {
-  static std::mutex mu;
-  static uint64_t done = 0;  // bit per device ordinal
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  const uint64_t bit = 1ull << dev;
-  std::lock_guard<std::mutex> lock(mu);
-  if (done & bit) return cudaSuccess;
-  cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, patch_attn_kernel<D, NQ>);
-  if (e != cudaSuccess) return e;
-  if (128 * static_cast<long>(kRegsOther) + 256 * static_cast<long>(kRegsSoftmax) >
-      static_cast<long>(kThreads) * fa.numRegs)
-    return cudaErrorNotSupported;  // the split would wait forever in setmaxnreg.inc
-  e = cudaFuncSetAttribute(patch_attn_kernel<D, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem_bytes<D, NQ>());
-  if (e != cudaSuccess) return e;
-  done |= bit;
-  return cudaSuccess;
-}
-
-template <int D, int NQ>
-cudaError_t launch_one(const AttnParams& p, cudaStream_t stream) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  e = configure_once<D, NQ>(dev);
-  if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.n_split);
-  patch_attn_kernel<D, NQ><<<grid, kThreads, smem_bytes<D, NQ>(), stream>>>(p);
-  return cudaGetLastError();
-}
-
 // ------------------------------------------------------------------ head_dim 64: half rows
 //
 // With head_dim 64 a key tile costs the tensor core half of what it costs at 128 while the
 // softmax still exponentiates 128 x 128 scores per query tile, so the exponentials, not the
 // MMAs, bound the loop; with one thread per query row there are only two softmax warps per
 // SM sub-partition to keep the special-function unit busy, and each runs a long dependent
-// chain.  This kernel splits every 128-key tile between two softmax warpgroups per query
-// tile: half 0 owns keys 0..63 of each tile, half 1 keys 64..127.  Each half is an
-// independent online softmax over its own keys, with its own reference maximum m, row sum
-// l and O accumulator in TMEM, so the halves never wait for each other inside the loop;
-// they are combined once per CTA, log-sum-exp style (O = (2^(m_0-M) O_0 + 2^(m_1-M) O_1) /
-// (2^(m_0-M) l_0 + 2^(m_1-M) l_1), M = max(m_0, m_1)).  Four softmax warps per
-// sub-partition instead of two.
+// chain.  Here every query row is shared by two threads: half 0 of a query tile's softmax
+// warps takes keys 0..63 of each key tile, half 1 keys 64..127, so four softmax warps run
+// per sub-partition.  The two threads of a row keep one reference maximum m (they exchange
+// their half-tile maxima through shared memory once per tile, behind a 64-thread barrier
+// that also carries their agreement on aborting), one O accumulator in TMEM (each half
+// rescales 32 of its 64 columns) and a row sum each, added once at the end.
 //
-// TMEM, per query tile t (256 columns at 256 t): S_0 | S_1 (64 fp32 columns each) | O_0 | O_1
-// (64 each).  P_h (packed bf16) is written over the first 32 columns of S_h, so QK_h(j+1)
-// is issued after PV_h(j) by the same thread; the tensor pipe completes in order, so
-// S_h(j+1) being complete also means PV_h(j) has read P_h(j) and finished O_h.
+// TMEM, per query tile t (256 columns at 256 t): S (128 fp32 columns) | O (64) | P_0 (32) |
+// P_1 (32): P (packed bf16) has its own columns, so QK(j+1) is issued (one N = 128 MMA
+// chain) as soon as every softmax warp of the tile has S(j) in registers and runs while
+// they exponentiate.  P(j) may overwrite P(j-1) only after PV(j-1) has read it: QK(j+1) was
+// issued by the same thread after PV(j-1), so S(j+1) being complete implies it (the last
+// tile waits for the PV itself).
 //
 // Warps: 0-15 softmax (warp w: query tile w / 8, half (w / 4) % 2, TMEM lane quarter w % 4),
 // 16 TMEM allocation + MMA issuer of query tile 0, 17 TMA producer, 18 scatter, 19 MMA
-// issuer of query tile 1.
+// issuer of query tile 1.  Named barriers: 1 + 4 t + quarter (the two warps of a row
+// quarter, 64 threads), 9 + t (the 256 softmax threads of query tile t).
 constexpr int kHrThreads = 640;
 constexpr int kHrLaunchRegs = (65536 / kHrThreads) / 8 * 8;  // 96
 constexpr uint32_t kHrRegsSoftmax = 104;
@@ -1002,6 +320,8 @@ constexpr int kHrWarpMma1 = 19;
 constexpr int kHrStages = 8;
 constexpr int kHrTile = kRows * 64 * 2;  // 16 KB: 128 rows x 64 bf16, one 128-byte swizzle span
 constexpr int kHrPoly = 2;               // of every 8 column pairs, exponentiated on the FMA pipe
+constexpr uint32_t kHrColO = 128;        // within a query tile's 256 columns
+constexpr uint32_t kHrColP = 192;
 
 template <int NQ>
 constexpr int hr_smem_bytes() {
@@ -1025,6 +345,30 @@ __device__ __forceinline__ float row_max64(const uint32_t (&s)[64]) {
   return max3(mv[0], mv[1], fmaxf(mv[2], mv[3]));
 }
 
+// p_k = 2^(s_k c - m) for 64 scores, packed to bf16 pairs, POLY of every 8 column pairs on
+// the FMA pipe; the fp32 sum goes to lsum.  With SPEC, also returns max_k (s_k c - m), so a
+// caller exponentiating against a reference that may be stale can check that no p_k exceeded
+// 2^8 (masked keys, -inf, are ignored by the maximum).
+template <int POLY, bool SPEC>
+__device__ __forceinline__ float exps64(const uint32_t (&s)[64], float c, float m, uint32_t (&pk)[32],
+                                        float& lsum) {
+  const float2 cc = make_float2(c, c), nm = make_float2(-m, -m);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
+  float xm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), cc, nm);
+    if (SPEC) xm[k & 3] = max3(xm[k & 3], x.x, x.y);
+    const float2 pe = (k & 7) < POLY ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
+    acc[k & 3] = __fadd2_rn(acc[k & 3], pe);
+    pk[k] = pack_bf16(pe.x, pe.y);
+  }
+  const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  lsum = a.x + a.y;
+  return SPEC ? fmaxf(fmaxf(xm[0], xm[1]), fmaxf(xm[2], xm[3])) : 0.f;
+}
+
 template <int NQ>
 __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __grid_constant__ AttnParams p) {
   constexpr int D = 64;
@@ -1038,14 +382,16 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + S;
-  uint64_t* s_full = kv_empty + S;  // [2 t + h]
-  uint64_t* p_full = s_full + 4;    // [2 t + h]
-  uint64_t* o_full = p_full + 4;    // [2 t + h]
-  uint64_t* mma_done = o_full + 4;  // [issuer]
+  uint64_t* s_full = kv_empty + S;  // [t]
+  uint64_t* s_free = s_full + 2;    // [t]: every softmax warp of the tile has S in registers
+  uint64_t* p_full = s_free + 2;    // [t]
+  uint64_t* pv_done = p_full + 2;   // [t]
+  uint64_t* o_full = pv_done + 2;   // [t]
+  uint64_t* mma_done = o_full + 2;  // [issuer]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  __shared__ float xch_m[2][2][kRows];  // [t][h][row]: each half's m and l for the combine
-  __shared__ float xch_l[2][2][kRows];
+  __shared__ float xch_m[2][2][2][kRows];  // [tile parity][t][half][row]: half-tile maxima
+  __shared__ float xch_l[2][2][kRows];     // [t][half][row]: row sums at the end
   __shared__ int s_last[2];
 
   PF_TRACE_CTA(1);
@@ -1066,13 +412,14 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
       mbar_init(smem_u32(kv_full + st), 1);
       mbar_init(smem_u32(kv_empty + st), NQ);  // one commit per MMA issuer (one per query tile)
     }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(smem_u32(s_full + i), 1);
-      mbar_init(smem_u32(p_full + i), 4);  // one arrival per softmax warp of the half
-      mbar_init(smem_u32(o_full + i), 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(smem_u32(s_full + t), 1);
+      mbar_init(smem_u32(s_free + t), 8);  // one arrival per softmax warp of the tile
+      mbar_init(smem_u32(p_full + t), 8);
+      mbar_init(smem_u32(pv_done + t), 1);
+      mbar_init(smem_u32(o_full + t), 1);
+      mbar_init(smem_u32(mma_done + t), 1);
     }
-    mbar_init(smem_u32(mma_done), 1);
-    mbar_init(smem_u32(mma_done + 1), 1);
     *abort = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -1104,6 +451,9 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the next micro-step may start its CTAs (set-up, Q and fresh K/V loads) on SMs this grid
+  // leaves idle; everything that touches memory this grid writes waits (grid_dep_wait)
+  grid_dep_launch();
 
   Segments seg;
   seg.init(p);
@@ -1123,9 +473,15 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
           tma_load_4d(smem_u32(sQ + t * kHrTile), &p.tm_q, 0, hd, q0 + t * kRows, b, qbar);
         int issued = 0;
         bool ok = true;
+        bool dep_done = false;
         for (int j = 0; j < n_tiles && ok; ++j) {
           int src, row0, nv;
           seg.tile(j0 + j, src, row0, nv);
+          if ((src == 1 || src == 3) && !dep_done) {
+            // buffer rows: the previous micro-step's scatter writes some of them
+            grid_dep_wait();
+            dep_done = true;
+          }
           for (int kv = 0; kv < 2; ++kv) {
             const int i = 2 * j + kv;
             const int st = i % S;
@@ -1153,28 +509,25 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
       // ------------------------------------------------------------ MMA issuer of query tile t
       if (lane == 0) {
         const int t = warp == kHrWarpMma0 ? 0 : 1;
-        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, 0);  // N = 64 keys, K-major K
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 64, 1);  // N = 64 columns, MN-major V
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0);  // N = 128 keys, K-major K
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 64, 1);   // N = 64 columns, MN-major V
         const uint32_t q_lo = ((smem_u32(sQ) + t * kHrTile) >> 4) | desc_lbo_bits(16);
         const uint32_t k_lo = (smem_u32(sKV) >> 4) | desc_lbo_bits(16);
         const uint32_t v_lo = (smem_u32(sKV) >> 4) | desc_lbo_bits(kChunkBytes);
-        // S_h = Q_t K[64 h .. 64 h + 63]^T: the half's 64 key rows start 64 * 128 bytes in
-        auto issue_qk = [=](int h, int st) {
-          const uint32_t b0 = k_lo + static_cast<uint32_t>((st * kHrTile + h * 8192) >> 4);
-          const uint32_t d = tmem + t * 256 + h * 64;
+        const uint32_t tbase = tmem + t * 256;
+        auto issue_qk = [=](int st) {
+          const uint32_t b0 = k_lo + static_cast<uint32_t>((st * kHrTile) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ss(d, smem_desc_lo(q_lo + 2 * kk), smem_desc_lo(b0 + 2 * kk), idesc_qk, kk > 0);
+            mma_ss(tbase, smem_desc_lo(q_lo + 2 * kk), smem_desc_lo(b0 + 2 * kk), idesc_qk, kk > 0);
         };
-        // O_h += P_h V[64 h .. 64 h + 63]: P_h from TMEM (over S_h), 16 keys per MMA
-        auto issue_pv = [=](int h, int st, bool acc) {
-          const uint32_t v0 = v_lo + static_cast<uint32_t>((st * kHrTile + h * 8192) >> 4);
-          const uint32_t d = tmem + t * 256 + 128 + h * 64;
-          const uint32_t a = tmem + t * 256 + h * 64;
+        // O += [P_0 | P_1] V: 16 keys per MMA, P from TMEM
+        auto issue_pv = [=](int st, bool acc) {
+          const uint32_t v0 = v_lo + static_cast<uint32_t>((st * kHrTile) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ts(d, a + kk * 8, smem_desc_lo(v0 + static_cast<uint32_t>((kk * 2048) >> 4)), idesc_pv,
-                   acc || kk > 0);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tbase + kHrColO, tbase + kHrColP + kk * 8,
+                   smem_desc_lo(v0 + static_cast<uint32_t>((kk * 2048) >> 4)), idesc_pv, acc || kk > 0);
         };
 
         bool ok = mbar_wait(smem_u32(q_full), 0, abort, kWaitNs);
@@ -1182,36 +535,34 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
           ok = mbar_wait(smem_u32(kv_full + 0), 0, abort, kWaitNs);  // K(0): load 0, stage 0
           tc_fence_after();
           if (ok) {
-            issue_qk(0, 0);
-            mma_commit(smem_u32(s_full + 2 * t));
-            issue_qk(1, 0);
-            mma_commit(smem_u32(s_full + 2 * t + 1));
+            issue_qk(0);
+            mma_commit(smem_u32(s_full + t));
             mma_commit(smem_u32(kv_empty + 0));
           }
         }
         for (int j = 0; j < n_tiles && ok; ++j) {
+          if (j + 1 < n_tiles) {
+            // QK(j+1) as soon as every softmax warp of the tile has S(j) in registers
+            const int iK = 2 * (j + 1), sK = iK % S;
+            if (!(ok = mbar_wait(smem_u32(kv_full + sK), (iK / S) & 1, abort, kWaitNs))) break;
+            if (!(ok = mbar_wait(smem_u32(s_free + t), j & 1, abort, kWaitNs))) break;
+            tc_fence_after();
+            PF_TRACE_AT(4, 2 * t, j);
+            issue_qk(sK);
+            mma_commit(smem_u32(s_full + t));
+            mma_commit(smem_u32(kv_empty + sK));
+            PF_TRACE_AT(3, 2 * t, j);
+          }
           const int iV = 2 * j + 1, sV = iV % S;
           if (!(ok = mbar_wait(smem_u32(kv_full + sV), (iV / S) & 1, abort, kWaitNs))) break;
-          const bool has_next = j + 1 < n_tiles;
-          const int iK = 2 * (j + 1), sK = iK % S;
-          if (has_next && !(ok = mbar_wait(smem_u32(kv_full + sK), (iK / S) & 1, abort, kWaitNs))) break;
-          PF_TRACE_AT(4, 2 * t, j);
-          for (int h = 0; h < 2; ++h) {
-            if (!(ok = mbar_wait(smem_u32(p_full + 2 * t + h), j & 1, abort, kWaitNs))) break;
-            tc_fence_after();
-            PF_TRACE_AT(2, 2 * t + h, j);
-            issue_pv(h, sV, j > 0);
-            if (has_next) {
-              issue_qk(h, sK);
-              mma_commit(smem_u32(s_full + 2 * t + h));
-            } else {
-              mma_commit(smem_u32(o_full + 2 * t + h));
-            }
-            PF_TRACE_AT(3, 2 * t + h, j);
-          }
-          if (!ok) break;
+          if (!(ok = mbar_wait(smem_u32(p_full + t), j & 1, abort, kWaitNs))) break;
+          tc_fence_after();
+          PF_TRACE_AT(2, 2 * t, j);
+          issue_pv(sV, j > 0);
+          mma_commit(smem_u32(pv_done + t));
           mma_commit(smem_u32(kv_empty + sV));
-          if (has_next) mma_commit(smem_u32(kv_empty + sK));
+          if (j + 1 == n_tiles) mma_commit(smem_u32(o_full + t));
+          PF_TRACE_AT(3, 2 * t + 1, j);
         }
         if (!ok) raise_abort(abort, kWdMma);
         // drain every MMA issued by this thread before TMEM is released
@@ -1228,12 +579,15 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
     const int t = warp >> 3;
     const int hh = (warp >> 2) & 1;
     const int wq = warp & 3;
+    const int pair_bar = 1 + 4 * t + wq;  // the two warps (halves) of this row quarter
+    const int rloc = wq * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + t * 256 + hh * 64;
-    const uint32_t tO = tmem + lane_off + t * 256 + 128 + hh * 64;
+    const uint32_t tO = tmem + lane_off + t * 256 + kHrColO + hh * 32;  // this half's 32 O columns
+    const uint32_t tP = tmem + lane_off + t * 256 + kHrColP + hh * 32;
     const float c = p.scale_log2;
-    float m = -INFINITY;  // this half's reference row maximum, in log2 units
-    float l = 0.f;
+    float m = -INFINITY;  // the row's reference maximum, in log2 units (same in both halves)
+    float l = 0.f;        // this half's part of the row sum
     bool ok = true;
     // local indices of this CTA's ragged context tiles and the valid keys of this half there
     int rag_j[4], rag_nv[4];
@@ -1249,10 +603,9 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
         rag_j[k] = (nv != 0 && e >= j0 && e < j1) ? e - j0 : -1;
       }
     }
+    bool s_ready = false;  // S(j) was seen complete at the end of tile j-1
     for (int j = 0; j < n_tiles; ++j) {
-      ok = mbar_wait(smem_u32(s_full + 2 * t + hh), j & 1, abort, kWaitNs);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
+      if (!s_ready) ok = ok && mbar_wait(smem_u32(s_full + t), j & 1, abort, kWaitNs);
       tc_fence_after();
       if (wq == 0 && lane == 0) PF_TRACE_AT(0, 2 * t + hh, j);
       uint32_t s[64];
@@ -1260,6 +613,10 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
       tmem_ld32(tS + 32, s + 32);
       tmem_wait_ld();
       reg_fence<64>(s);
+      // S is in registers: hand its columns back so QK(j+1) can start
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(s_free + t));
       int nv = 64;
 #pragma unroll
       for (int k = 0; k < 4; ++k)
@@ -1269,18 +626,57 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
         for (int k = 0; k < 64; ++k)
           if (k >= nv) s[k] = __float_as_uint(-INFINITY);
       }
-      const float mxs = row_max64(s) * c;
+      // the row maximum over both halves: exchange, behind a barrier that also makes the two
+      // warps agree on going on (a warp whose wait failed must not leave its partner waiting)
+      xch_m[j & 1][t][hh][rloc] = row_max64(s);
+      ok = named_bar_and(pair_bar, 64, ok);
+      if (!ok) break;
+      const float mxs = fmaxf(xch_m[j & 1][t][0][rloc], xch_m[j & 1][t][1][rloc]) * c;
       if (wq == 0 && lane == 0) PF_TRACE_AT(6, 2 * t + hh, j);
-      const bool grow = mxs > m + 8.f;
+      const bool grow = mxs > m + 8.f;  // the same decision in both halves
       // warp-collective TMEM accesses: the whole warp rescales when any of its rows grew
-      // (alpha is exactly 1 for the others).  S_h(j) being complete means PV_h(j-1) is too.
+      // (alpha is exactly 1 for the others)
       const bool any_grow = __any_sync(0xffffffffu, grow);
       const float alpha = grow ? ex2(m - mxs) : 1.f;
       l *= alpha;
       m = grow ? mxs : m;
-      if (any_grow && j > 0) {
+      // P(j) may overwrite P(j-1) once PV(j-1) has read it: S(j+1) complete implies it (QK(j+1)
+      // was issued after PV(j-1)); the last tile waits for PV(j-1) itself.  Probed half way
+      // through the exponentials so the wait is usually over.
+      const bool has_next = j + 1 < n_tiles;
+      const uint32_t gate = has_next ? smem_u32(s_full + t) : smem_u32(pv_done + t);
+      const uint32_t gate_par = has_next ? static_cast<uint32_t>((j + 1) & 1)
+                                         : static_cast<uint32_t>((j - 1) & 1);
+      bool gate_ok = !has_next && j == 0;  // a single tile: nothing to wait for
+      uint32_t pk[32];
+      {
+        const float2 cc = make_float2(c, c), nm = make_float2(-m, -m);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 16) {
+        for (int k = 0; k < 32; ++k) {
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), cc, nm);
+          const float2 pe = (k & 7) < kHrPoly ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
+          acc[k & 3] = __fadd2_rn(acc[k & 3], pe);
+          pk[k] = pack_bf16(pe.x, pe.y);
+          if (k == 15 && !gate_ok) gate_ok = mbar_test_wait_all(gate, gate_par);
+        }
+        const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+        l += a.x + a.y;
+      }
+      if (wq == 0 && lane == 0) PF_TRACE_AT(7, 2 * t + hh, j);
+      if (!gate_ok) {
+        // on failure go on (the abort flag is up): the partner learns of it at the next
+        // exchange, and both leave the loop together
+        if (!mbar_wait(gate, gate_par, abort, kWaitNs)) ok = false;
+        ok = __all_sync(0xffffffffu, ok);
+      }
+      tc_fence_after();
+      s_ready = has_next;
+      if (any_grow && j > 0) {
+        // this half rescales its 32 of the row's 64 O columns (PV(j-1) is complete)
+#pragma unroll
+        for (int c0 = 0; c0 < 32; c0 += 16) {
           uint32_t o[16];
           tmem_ld16(tO + c0, o);
           tmem_wait_ld();
@@ -1290,69 +686,40 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
           tmem_st16(tO + c0, o);
         }
       }
-      // a half-row with no valid key so far (its keys all masked) exponentiates against 0:
-      // masked keys then give 0 (or 2^-125 on the polynomial) instead of NaN
-      const float mref = m == -INFINITY ? 0.f : m;
-      uint32_t pk[32];
-      {
-        const float2 cc = make_float2(c, c), nm = make_float2(-mref, -mref);
-        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                         make_float2(0.f, 0.f)};
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), cc, nm);
-          const float2 pe = (k & 7) < kHrPoly ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
-          acc[k & 3] = __fadd2_rn(acc[k & 3], pe);
-          pk[k] = pack_bf16(pe.x, pe.y);
-        }
-        const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-        l += a.x + a.y;
-      }
-      if (wq == 0 && lane == 0) PF_TRACE_AT(7, 2 * t + hh, j);
-      tmem_st32(tS, pk);
+      tmem_st32(tP, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(p_full + 2 * t + hh));
+      if (lane == 0) mbar_arrive(smem_u32(p_full + t));
       if (wq == 0 && lane == 0) PF_TRACE_AT(1, 2 * t + hh, j);
     }
     if (!ok && lane == 0) raise_abort(abort, kWdSoftmax);
     {
-      bool ok_o = ok && mbar_wait(smem_u32(o_full + 2 * t + hh), 0, abort, kWaitNs);
+      bool ok_o = ok && mbar_wait(smem_u32(o_full + t), 0, abort, kWaitNs);
       ok_o = __all_sync(0xffffffffu, ok_o);
-      // both halves of the query tile take the same branch (the combine has barriers)
-      ok_o = named_bar_and(1 + t, 2 * kRows, ok_o);
+      // both halves of the query tile take the same branch (the epilogue has barriers)
+      ok_o = named_bar_and(9 + t, 2 * kRows, ok_o);
       if (!ok_o) {
         if (ok && lane == 0) raise_abort(abort, kWdEpilogue);
       } else {
         tc_fence_after();
-        const int rloc = wq * 32 + lane;
+        grid_dep_wait();  // the output and the workspace may be in use by the previous grid
         const int row = q0 + t * kRows + rloc;
         const bool in_range = row < p.q_rows;
-        // combine the two halves of the row: this thread produces columns 32 hh .. 32 hh + 31
-        xch_m[t][hh][rloc] = m;
         xch_l[t][hh][rloc] = l;
-        named_bar_sync(1 + t, 2 * kRows);
-        const float m_o = xch_m[t][hh ^ 1][rloc];
-        const float l_o = xch_l[t][hh ^ 1][rloc];
-        const float mrow = fmaxf(m, m_o);  // finite: half 0 has a valid key in every tile
-        const float w_me = ex2(m - mrow), w_o = ex2(m_o - mrow);
-        const float lrow = w_me * l + w_o * l_o;
-        const float w0 = hh == 0 ? w_me : w_o, w1 = hh == 0 ? w_o : w_me;
-        const uint32_t tO0 = tmem + lane_off + t * 256 + 128 + hh * 32;  // O_0 columns of this thread
+        named_bar_sync(9 + t, 2 * kRows);
+        const float lrow = xch_l[t][0][rloc] + xch_l[t][1][rloc];
         float o[32];
 #pragma unroll
         for (int c0 = 0; c0 < 32; c0 += 16) {
-          uint32_t a0[16], a1[16];
-          tmem_ld16(tO0 + c0, a0);
-          tmem_ld16(tO0 + 64 + c0, a1);
+          uint32_t a0[16];
+          tmem_ld16(tO + c0, a0);
           tmem_wait_ld();
           reg_fence<16>(a0);
-          reg_fence<16>(a1);
 #pragma unroll
-          for (int k = 0; k < 16; ++k)
-            o[c0 + k] = w0 * __uint_as_float(a0[k]) + w1 * __uint_as_float(a1[k]);
+          for (int k = 0; k < 16; ++k) o[c0 + k] = __uint_as_float(a0[k]);
         }
+        // this thread's 32 output columns: 32 hh .. 32 hh + 31
         uint16_t* dst = p.o + ((static_cast<size_t>(b) * p.q_rows + row) * p.heads + hd) * D + 32 * hh;
         if (p.n_split == 1) {
           const float inv = 1.f / lrow;
@@ -1375,11 +742,11 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
 #pragma unroll
           for (int k = 0; k < 32; ++k) mine[(32 * hh + k) * kRows + rloc] = o[k];
           if (hh == 0) {
-            mine[D * kRows + rloc] = mrow;
+            mine[D * kRows + rloc] = m;
             mine[(D + 1) * kRows + rloc] = lrow;
           }
           __threadfence();
-          named_bar_sync(1 + t, 2 * kRows);
+          named_bar_sync(9 + t, 2 * kRows);
           if (hh == 0 && rloc == 0) {
             const unsigned old = atomicAdd(p.ws_cnt + pair * 2 + t, 1u);
             const int last = old == static_cast<unsigned>(p.n_split - 1);
@@ -1389,7 +756,7 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
             }
             s_last[t] = last;
           }
-          named_bar_sync(1 + t, 2 * kRows);
+          named_bar_sync(9 + t, 2 * kRows);
           if (s_last[t]) {
             // merge every part of this query tile: this thread's 32 columns of its row
             float mref = -INFINITY, lsum = 0.f;
@@ -1443,6 +810,26 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
   }
 }
 
+// Launch an attention kernel with programmatic stream serialization: when the previous
+// work on the stream is another attention launch, this grid's CTAs may start while that one
+// finishes (it signals with grid_dep_launch); the kernel waits (grid_dep_wait) before it
+// reads the K/V buffer or writes the buffer, the output or the workspace.  After any other
+// kind of work the launch simply waits for it, as an ordinary launch does.
+cudaError_t launch_overlapped(void (*kernel)(AttnParams), const AttnParams& p, int threads, int smem,
+                              cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.n_split));
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 template <int NQ>
 cudaError_t hr_configure_once(int dev) {
   static std::mutex mu;
@@ -1471,9 +858,7 @@ cudaError_t launch_hr(const AttnParams& p, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   e = hr_configure_once<NQ>(dev);
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.n_split);
-  patch_attn_hr_kernel<NQ><<<grid, kHrThreads, hr_smem_bytes<NQ>(), stream>>>(p);
-  return cudaGetLastError();
+  return launch_overlapped(patch_attn_hr_kernel<NQ>, p, kHrThreads, hr_smem_bytes<NQ>(), stream);
 }
 
 // Epilogue of a softmax thread that owns a whole query row: O (TMEM columns from tO) over l
@@ -1676,6 +1061,9 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the next micro-step may start its CTAs (set-up, Q and fresh K/V loads) on SMs this grid
+  // leaves idle; everything that touches memory this grid writes waits (grid_dep_wait)
+  grid_dep_launch();
 
   Segments seg;
   seg.init(p);
@@ -1697,9 +1085,15 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
                         q0 + t * kRows, b, qbar);
         int issued = 0;
         bool ok = true;
+        bool dep_done = false;
         for (int j = 0; j < n_tiles && ok; ++j) {
           int src, row0, nv;
           seg.tile(j0 + j, src, row0, nv);
+          if ((src == 1 || src == 3) && !dep_done) {
+            // buffer rows: the previous micro-step's scatter writes some of them
+            grid_dep_wait();
+            dep_done = true;
+          }
           for (int kv = 0; kv < 2; ++kv) {
             const int i = 2 * j + kv;
             const int st = i % S;
@@ -1849,49 +1243,61 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
           for (int k = 0; k < 64; ++k)
             if (k >= nvh) s[k] = __float_as_uint(-INFINITY);
         }
-        const float mxs = row_max64(s) * c;
-        const bool grow = mxs > m + 8.f;
-        // warp-collective TMEM accesses: the whole warp rescales when any of its rows grew
-        // (alpha is exactly 1 for the others)
-        const bool any_grow = __any_sync(0xffffffffu, grow);
-        const float alpha = grow ? ex2(m - mxs) : 1.f;
-        if (any_grow && (j > 0 || h > 0)) {
-          // O holds earlier PVs: PV_h(j-1) is complete (S_h(j) is); wait for the other
-          // half's latest one, PV_1(j-1) before half 0, PV_0(j) before half 1
-          const uint32_t par = h == 0 ? static_cast<uint32_t>((j - 1) & 1) : static_cast<uint32_t>(j & 1);
-          ok = mbar_wait(smem_u32(pv_done + 2 * t + (h ^ 1)), par, abort, kWaitNs);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
-            uint32_t o[16];
-            tmem_ld16(tO + c0, o);
-            tmem_wait_ld();
-            reg_fence<16>(o);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st16(tO + c0, o);
-          }
-        }
-        l *= alpha;
-        m = grow ? mxs : m;
-        const float mref = m == -INFINITY ? 0.f : m;  // no valid key yet: masked keys give 0
+        // Fast path: exponentiate against the current reference maximum straight away and
+        // check afterwards that no value exceeded 2^8, so the row maximum is off the critical
+        // path.  The CTA's first half-tile (no reference yet: m is -inf in every row) and the
+        // rare half whose maximum grew by more than 2^8 take the exact path.
         uint32_t pk[32];
-        {
-          const float2 cc = make_float2(c, c), nm = make_float2(-mref, -mref);
-          float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                           make_float2(0.f, 0.f)};
+        float lsum;
+        bool exact = m == -INFINITY;
+        if (!exact) {
+          const float xm = exps64<kPolyPairs<D>, true>(s, c, m, pk, lsum);
+          // warp-uniform decision (the reload is a warp-collective TMEM access)
+          if (__any_sync(0xffffffffu, xm > 8.f)) {
+            // S_h is still in TMEM (P_h has not been written yet): reload it
+            exact = true;
+            tmem_ld32(tS + h * 64, s);
+            tmem_ld32(tS + h * 64 + 32, s + 32);
+            tmem_wait_ld();
+            reg_fence<64>(s);
+            if (nvh < 64) {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), cc, nm);
-            const float2 pe = (k & 7) < kPolyPairs<D> ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
-            acc[k & 3] = __fadd2_rn(acc[k & 3], pe);
-            pk[k] = pack_bf16(pe.x, pe.y);
+              for (int k = 0; k < 64; ++k)
+                if (k >= nvh) s[k] = __float_as_uint(-INFINITY);
+            }
           }
-          const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-          l += a.x + a.y;
         }
+        if (exact) {
+          const float mxs = row_max64(s) * c;
+          const bool grow = mxs > m + 8.f;
+          // warp-collective TMEM accesses: the whole warp rescales when any of its rows grew
+          // (alpha is exactly 1 for the others)
+          const bool any_grow = __any_sync(0xffffffffu, grow);
+          const float alpha = grow ? ex2(m - mxs) : 1.f;
+          if (any_grow && (j > 0 || h > 0)) {
+            // O holds earlier PVs: PV_h(j-1) is complete (S_h(j) is); wait for the other
+            // half's latest one, PV_1(j-1) before half 0, PV_0(j) before half 1
+            const uint32_t par = h == 0 ? static_cast<uint32_t>((j - 1) & 1) : static_cast<uint32_t>(j & 1);
+            ok = mbar_wait(smem_u32(pv_done + 2 * t + (h ^ 1)), par, abort, kWaitNs);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int c0 = 0; c0 < Dm::kMmaN; c0 += 16) {
+              uint32_t o[16];
+              tmem_ld16(tO + c0, o);
+              tmem_wait_ld();
+              reg_fence<16>(o);
+#pragma unroll
+              for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+              tmem_st16(tO + c0, o);
+            }
+          }
+          l *= alpha;
+          m = grow ? mxs : m;
+          exps64<kPolyPairs<D>, false>(s, c, m, pk, lsum);
+        }
+        l += lsum;
         if (wq == 0 && lane == 0) PF_TRACE_AT(7, 2 * t + h, j);
         tmem_st32(tS + h * 64, pk);
         tmem_wait_st();
@@ -1911,6 +1317,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
         if (ok && lane == 0) raise_abort(abort, kWdEpilogue);
       } else {
         tc_fence_after();
+        grid_dep_wait();  // the output and the workspace may be in use by the previous grid
         full_row_epilogue<D>(p, tO, m, l, pair, part, t, q0, hd, b, wq, lane, s_last);
       }
     }
@@ -1956,9 +1363,7 @@ cudaError_t launch_sn(const AttnParams& p, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   e = sn_configure_once<D, NQ>(dev);
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.n_split);
-  patch_attn_sn_kernel<D, NQ><<<grid, kThreads, smem_bytes<D, NQ>(), stream>>>(p);
-  return cudaGetLastError();
+  return launch_overlapped(patch_attn_sn_kernel<D, NQ>, p, kThreads, smem_bytes<D, NQ>(), stream);
 }
 
 __global__ void zero_u32_kernel(unsigned* p, size_t n) {
