@@ -743,6 +743,19 @@ def run_profile_calls(args):
     return 0
 
 
+def run_profile_norm(args):
+    """For ncu captures: two per-head RMS normalisations of a full-spatial Q of the workload."""
+    import patch_attention_b200 as pa
+
+    wl = synth.ATTN_WORKLOADS[args.workload]
+    g = torch.Generator(device="cuda").manual_seed(5)
+    x = torch.randn(wl.batch, wl.n_img, wl.heads, wl.head_dim, device="cuda", generator=g).bfloat16()
+    for _ in range(2):
+        pa.pf_qk_rmsnorm(x)
+    torch.cuda.synchronize()
+    return 0
+
+
 def run_profile_cfg(args):
     """For ncu captures: two guidance-kernel calls at the largest sweep size."""
     import patch_attention_b200 as pa
@@ -761,6 +774,8 @@ def main():
                     help="only run the start-up pass and this many micro-steps of one layer (for ncu)")
     ap.add_argument("--profile-cfg", action="store_true",
                     help="only run two guidance-kernel calls at the largest size (for ncu)")
+    ap.add_argument("--profile-norm", action="store_true",
+                    help="only run two RMS normalisations of a full-spatial Q of the workload (for ncu)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
@@ -778,6 +793,8 @@ def main():
         return run_profile_calls(args)
     if args.profile_cfg:
         return run_profile_cfg(args)
+    if args.profile_norm:
+        return run_profile_norm(args)
     world, rank, local = dist_setup()
     try:
         if args.impl == "reference":

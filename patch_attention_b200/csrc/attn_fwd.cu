@@ -60,7 +60,7 @@ constexpr int kTraceTiles = 512;
 // 9 MMA issuer sees the V tile of j-1, 10 producer issued the K (t=0) / V (t=1) tile j.
 // The second index is the softmax chain: the query tile (full-row kernels) or 2 * query tile
 // + key half (half-row kernel).
-__device__ unsigned long long g_trace[11 * 4 * kTraceTiles];
+__device__ unsigned long long g_trace[16 * 4 * kTraceTiles];
 // Per CTA of the latest launch: SM id, start and end (global timer, ns).
 constexpr int kTraceCtas = 4096;
 __device__ unsigned long long g_cta[3 * kTraceCtas];
@@ -319,7 +319,7 @@ constexpr int kHrWarpScatter = 18;
 constexpr int kHrWarpMma1 = 19;
 constexpr int kHrStages = 8;
 constexpr int kHrTile = kRows * 64 * 2;  // 16 KB: 128 rows x 64 bf16, one 128-byte swizzle span
-constexpr int kHrPoly = 2;               // of every 8 column pairs, exponentiated on the FMA pipe
+constexpr int kHrPoly = 0;               // of every 8 column pairs, exponentiated on the FMA pipe
 constexpr uint32_t kHrColO = 128;        // within a query tile's 256 columns
 constexpr uint32_t kHrColP = 192;
 
@@ -346,27 +346,23 @@ __device__ __forceinline__ float row_max64(const uint32_t (&s)[64]) {
 }
 
 // p_k = 2^(s_k c - m) for 64 scores, packed to bf16 pairs, POLY of every 8 column pairs on
-// the FMA pipe; the fp32 sum goes to lsum.  With SPEC, also returns max_k (s_k c - m), so a
-// caller exponentiating against a reference that may be stale can check that no p_k exceeded
-// 2^8 (masked keys, -inf, are ignored by the maximum).
-template <int POLY, bool SPEC>
-__device__ __forceinline__ float exps64(const uint32_t (&s)[64], float c, float m, uint32_t (&pk)[32],
-                                        float& lsum) {
+// the FMA pipe; the fp32 sum goes to lsum.  Masked keys (-inf) give 0 on the special-function
+// unit and 2^-125 on the polynomial.
+template <int POLY>
+__device__ __forceinline__ void exps64(const uint32_t (&s)[64], float c, float m, uint32_t (&pk)[32],
+                                       float& lsum) {
   const float2 cc = make_float2(c, c), nm = make_float2(-m, -m);
   float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                    make_float2(0.f, 0.f)};
-  float xm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
   for (int k = 0; k < 32; ++k) {
     const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), cc, nm);
-    if (SPEC) xm[k & 3] = max3(xm[k & 3], x.x, x.y);
     const float2 pe = (k & 7) < POLY ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
     acc[k & 3] = __fadd2_rn(acc[k & 3], pe);
     pk[k] = pack_bf16(pe.x, pe.y);
   }
   const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
   lsum = a.x + a.y;
-  return SPEC ? fmaxf(fmaxf(xm[0], xm[1]), fmaxf(xm[2], xm[3])) : 0.f;
 }
 
 template <int NQ>
@@ -613,10 +609,12 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
       tmem_ld32(tS + 32, s + 32);
       tmem_wait_ld();
       reg_fence<64>(s);
+      if (wq == 0 && lane == 0) PF_TRACE_AT(5, 2 * t + hh, j);
       // S is in registers: hand its columns back so QK(j+1) can start
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(s_free + t));
+      if (wq == 0 && lane == 0) PF_TRACE_AT(10, 2 * t + hh, j);
       int nv = 64;
 #pragma unroll
       for (int k = 0; k < 4; ++k)
@@ -626,9 +624,13 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
         for (int k = 0; k < 64; ++k)
           if (k >= nv) s[k] = __float_as_uint(-INFINITY);
       }
+      if (wq == 0 && lane == 0) PF_TRACE_AT(11, 2 * t + hh, j);
+      const float mx_half = row_max64(s);
+      if (wq == 0 && lane == 0) PF_TRACE_AT(12, 2 * t + hh, j);
       // the row maximum over both halves: exchange, behind a barrier that also makes the two
       // warps agree on going on (a warp whose wait failed must not leave its partner waiting)
-      xch_m[j & 1][t][hh][rloc] = row_max64(s);
+      xch_m[j & 1][t][hh][rloc] = mx_half;
+      if (wq == 0 && lane == 0) PF_TRACE_AT(8, 2 * t + hh, j);
       ok = named_bar_and(pair_bar, 64, ok);
       if (!ok) break;
       const float mxs = fmaxf(xch_m[j & 1][t][0][rloc], xch_m[j & 1][t][1][rloc]) * c;
@@ -637,9 +639,12 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
       // warp-collective TMEM accesses: the whole warp rescales when any of its rows grew
       // (alpha is exactly 1 for the others)
       const bool any_grow = __any_sync(0xffffffffu, grow);
-      const float alpha = grow ? ex2(m - mxs) : 1.f;
-      l *= alpha;
-      m = grow ? mxs : m;
+      float alpha = 1.f;
+      if (any_grow) {
+        alpha = grow ? ex2(m - mxs) : 1.f;
+        l *= alpha;
+        m = grow ? mxs : m;
+      }
       // P(j) may overwrite P(j-1) once PV(j-1) has read it: S(j+1) complete implies it (QK(j+1)
       // was issued after PV(j-1)); the last tile waits for PV(j-1) itself.  Probed half way
       // through the exponentials so the wait is usually over.
@@ -672,6 +677,7 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
         ok = __all_sync(0xffffffffu, ok);
       }
       tc_fence_after();
+      if (wq == 0 && lane == 0) PF_TRACE_AT(9, 2 * t + hh, j);
       s_ready = has_next;
       if (any_grow && j > 0) {
         // this half rescales its 32 of the row's 64 O columns (PV(j-1) is complete)
@@ -1243,31 +1249,9 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
           for (int k = 0; k < 64; ++k)
             if (k >= nvh) s[k] = __float_as_uint(-INFINITY);
         }
-        // Fast path: exponentiate against the current reference maximum straight away and
-        // check afterwards that no value exceeded 2^8, so the row maximum is off the critical
-        // path.  The CTA's first half-tile (no reference yet: m is -inf in every row) and the
-        // rare half whose maximum grew by more than 2^8 take the exact path.
         uint32_t pk[32];
         float lsum;
-        bool exact = m == -INFINITY;
-        if (!exact) {
-          const float xm = exps64<kPolyPairs<D>, true>(s, c, m, pk, lsum);
-          // warp-uniform decision (the reload is a warp-collective TMEM access)
-          if (__any_sync(0xffffffffu, xm > 8.f)) {
-            // S_h is still in TMEM (P_h has not been written yet): reload it
-            exact = true;
-            tmem_ld32(tS + h * 64, s);
-            tmem_ld32(tS + h * 64 + 32, s + 32);
-            tmem_wait_ld();
-            reg_fence<64>(s);
-            if (nvh < 64) {
-#pragma unroll
-              for (int k = 0; k < 64; ++k)
-                if (k >= nvh) s[k] = __float_as_uint(-INFINITY);
-            }
-          }
-        }
-        if (exact) {
+        {
           const float mxs = row_max64(s) * c;
           const bool grow = mxs > m + 8.f;
           // warp-collective TMEM accesses: the whole warp rescales when any of its rows grew
@@ -1295,7 +1279,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
           }
           l *= alpha;
           m = grow ? mxs : m;
-          exps64<kPolyPairs<D>, false>(s, c, m, pk, lsum);
+          exps64<kPolyPairs<D>>(s, c, m, pk, lsum);
         }
         l += lsum;
         if (wq == 0 && lane == 0) PF_TRACE_AT(7, 2 * t + h, j);
