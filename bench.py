@@ -363,6 +363,11 @@ class StepRunner:
         self.pat.close()
 
 
+def attn_kernel_name(wl) -> str:
+    """The library's attention kernel for the workload's head_dim."""
+    return "patch_attn_hr_kernel" if wl.head_dim == 64 else "patch_attn_sn_kernel"
+
+
 def per_clock(tflops, clock_info, sms):
     """FLOP per SM per clock at the median SM clock of the timed region, and its fraction
     of the nominal dense bf16 rate (8192 FLOP/clk/SM)."""
@@ -373,7 +378,7 @@ def per_clock(tflops, clock_info, sms):
 
 
 def attn_roofline(wl, attn_ms, timed_s, peaks, peak_src, clock_info, sms, traffic):
-    """Roofline of patch_attn_kernel: algorithmic FLOP per launch / average launch time
+    """Roofline of the attention kernel: algorithmic FLOP per launch / average launch time
     (events around each step's attention section, launch gaps included).  The peak is the
     measured sustained bf16 rate when the timed region lasts at least 2 s, else the burst."""
     launch_ms = attn_ms / (wl.n_patches * wl.n_layers)
@@ -382,7 +387,7 @@ def attn_roofline(wl, attn_ms, timed_s, peaks, peak_src, clock_info, sms, traffi
     key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
     peak = float(peaks.get(key, peaks.get("bf16_tflops")))
     fpc, fpc_frac = per_clock(achieved, clock_info, sms)
-    return {"bound": "tensor", "kernel": "patch_attn_kernel", "achieved": achieved, "peak": peak,
+    return {"bound": "tensor", "kernel": attn_kernel_name(wl), "achieved": achieved, "peak": peak,
             "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
             "peak_source": f"{peak_src} {key} ({'timed region >= 2 s' if sustained else 'timed region < 2 s'})",
             "launch_ms": launch_ms, "flop_per_launch": wl.flop_per_call(),
@@ -484,7 +489,7 @@ def scatter_record(wl, traffic):
     """The fresh-K/V scatter is fused into the attention launch: its algorithmic bytes per
     call (K_p and V_p read and written), and their share of the launch's DRAM traffic."""
     b = 2 * 2 * wl.batch * wl.patch_len * wl.heads * wl.head_dim * 2
-    rec = {"bytes_per_call": b, "fused_into": "patch_attn_kernel",
+    rec = {"bytes_per_call": b, "fused_into": attn_kernel_name(wl),
            "launch_dram_bytes": traffic, "share_of_launch_dram": (b / traffic) if traffic else None}
     return rec
 
