@@ -284,6 +284,19 @@ __device__ __forceinline__ void scatter_share(const AttnParams& p, int lane) {
   }
 }
 
+// After the merge, the partial slots of a query tile ([part][d + 2][128] fp32) are dead: the next launch writes every slot before it reads one.  Dropping their L2 lines
+// keeps them from being written back to DRAM.  `tid` / `nthreads` split the lines among the
+// merging threads.
+template <int D>
+__device__ __forceinline__ void discard_partials(const float* slot0, int n_split, int tid, int nthreads) {
+  static_assert((D + 2) * kRows * 4 % 128 == 0, "slots are whole 128-byte lines");
+  const char* base = reinterpret_cast<const char*>(slot0);
+  // the workspace only has to be 16-byte aligned: skip when the lines are not whole
+  if ((reinterpret_cast<uintptr_t>(base) & 127u) != 0) return;
+  const int lines = n_split * (D + 2) * kRows * 4 / 128;
+  for (int i = tid; i < lines; i += nthreads) discard_l2_line(base + static_cast<size_t>(i) * 128);
+}
+
 // ------------------------------------------------------------------ head_dim 64: half rows
 //
 // With head_dim 64 a key tile costs the tensor core half of what it costs at 128 while the
@@ -798,6 +811,9 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
                 *reinterpret_cast<uint4*>(dst + k) = w;
               }
             }
+            // every thread of the tile has read all parts' slots: drop them from L2
+            named_bar_sync(9 + t, 2 * kRows);
+            discard_partials<D>(slot0, p.n_split, hh * kRows + rloc, 2 * kRows);
           }
         }
       }
@@ -966,6 +982,9 @@ __device__ __forceinline__ void full_row_epilogue(const AttnParams& p, uint32_t 
       }
     }
   }
+  // every thread of the tile has read all parts' slots: drop them from L2
+  named_bar_sync(1 + t, kRows);
+  discard_partials<D>(slot0, p.n_split, rloc, kRows);
 }
 
 // ------------------------------------------------------------------ head_dim 72/128: split key tiles

@@ -1,0 +1,63 @@
+"""Micro-steps launched back to back, with no host synchronisation between them.
+
+Consecutive attention launches overlap on the GPU (a launch's CTAs may start while the
+previous micro-step finishes and wait before they touch the K/V buffer, the output or the
+workspace).  The other parity tests synchronise after every call to check the buffer; here
+every call of a few diffusion steps is enqueued first, each into its own output, and only then
+checked: sampled rows of every call against the fp64 oracle, the buffer against the last step,
+and the device status word (a bounded wait that gave up would show as PF_ERR_TIMEOUT).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import patch_attention_b200 as pa
+from patch_attention_b200 import synth
+from tests._oracle_util import f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("d", [64, 72, 128])
+def test_overlapped_micro_steps_match_the_oracle(d):
+    wl = synth.AttnWorkload("b2b", batch=1, heads=4, head_dim=d, grid_h=64, grid_w=64,
+                            n_patches=8, n_txt=77, n_layers=2, n_steps=3, ar_a=0.95, ar_b=0.3)
+    S, L, M, P = wl.n_steps, wl.n_layers, wl.n_patches, wl.patch_len
+    gen = synth.AttnInputs(wl, seed=21, device="cuda")
+    steps = [[gen.step_tensors(l) for l in range(L)] for _ in range(S)]
+    pat = pa.PatchAttention(1, wl.heads, d, wl.n_img, M, wl.n_txt, L)
+    outs = {}
+    try:
+        for l in range(L):
+            pat.init_layer(l, steps[0][l]["k"], steps[0][l]["v"])
+        patches = [[[(t["q"][:, p * P:(p + 1) * P].contiguous(), t["k"][:, p * P:(p + 1) * P].contiguous(),
+                      t["v"][:, p * P:(p + 1) * P].contiguous()) for p in range(M)] for t in st] for st in steps]
+        torch.cuda.synchronize()
+        # every call of every step, in the pipeline's order, without a synchronisation
+        for s in range(S):
+            for p in range(M):
+                for l in range(L):
+                    q, k, v = patches[s][l][p]
+                    t = steps[s][l]
+                    outs[(s, l, p)] = pat.step(l, p, q, k, v, t["k_txt"], t["v_txt"])
+        torch.cuda.synchronize()
+        pat.check()  # no bounded wait gave up
+        rng = np.random.default_rng(3)
+        for (s, l, p), o in outs.items():
+            cur, prev = steps[s][l], steps[max(s - 1, 0)][l]
+            rows = sorted(set([0, P - 1] + list(rng.integers(0, P, 6))))
+            h = int(rng.integers(0, wl.heads))
+            take = lambda x: f64(x[0][:, h:h + 1])
+            ref = oracle.patch_attention(take(cur["q"]), take(cur["k"]), take(cur["v"]), take(prev["k"]),
+                                         take(prev["v"]), take(cur["k_txt"]), take(cur["v_txt"]), p, M,
+                                         wl.softmax_scale, rows=rows)
+            got = f64(o[0][rows][:, h:h + 1])
+            rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+            assert rel <= 5e-3, (s, l, p, rel)
+        for l in range(L):
+            kb, vb = pat.buffer_kv(l)
+            assert torch.equal(kb.view(torch.int16), steps[-1][l]["k"].view(torch.int16))
+            assert torch.equal(vb.view(torch.int16), steps[-1][l]["v"].view(torch.int16))
+    finally:
+        pat.close()
