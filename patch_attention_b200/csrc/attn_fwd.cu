@@ -77,7 +77,18 @@ __device__ unsigned long long g_cta[3 * kTraceCtas];
   do {                                                                                     \
     if (blockIdx.x == 0 && (j) < kTraceTiles) g_trace[((ev) * 4 + (t)) * kTraceTiles + (j)] = clock64(); \
   } while (0)
+// Per CTA, seen by thread 0 (a softmax thread of query tile 0), global timer ns: 0 set-up
+// done, 1 S of the first context tile seen, 2 O complete, 3 partial stored and fenced, 4
+// the last part is known, 5 merge done.
+__device__ unsigned long long g_cta_ev[8 * kTraceCtas];
+#define PF_TRACE_EV(slot)                                                                  \
+  do {                                                                                     \
+    if (threadIdx.x == 0 && blockIdx.x < kTraceCtas) g_cta_ev[8 * blockIdx.x + (slot)] = globaltimer_ns(); \
+  } while (0)
 #else
+#define PF_TRACE_EV(slot) \
+  do {                    \
+  } while (0)
 #define PF_TRACE_AT(ev, t, j) \
   do {                        \
   } while (0)
@@ -191,6 +202,88 @@ __device__ __forceinline__ void store_row16(uint16_t* dst, int c0, const uint32_
   }
 }
 
+// Merging the key-range parts of one query row.  Part i's slot holds, column-major with
+// kRows rows per column, the unnormalised O row (d columns) and then m_i and l_i; row0
+// points at this row's entry of part 0's slot.  The merged row is
+//   O = sum_i 2^(m_i - mref) O_i / sum_i 2^(m_i - mref) l_i,   mref = max_i m_i
+// (log-sum-exp combination of softmax parts).  The slots sit in L2, written by other CTAs,
+// so the merge is bound by L2 round trips: loads are issued for four parts at a time (and
+// for the O row, a block of columns of all four) before any of them is used.
+constexpr int kMergeGroup = 4;
+
+__device__ __forceinline__ void merge_stats(const float* row0, size_t slot_elems, int d, int n_split,
+                                            float& mref, float& inv) {
+  float mr = -INFINITY, ls = 0.f;
+  for (int i0 = 0; i0 < n_split; i0 += kMergeGroup) {
+    float mv[kMergeGroup], lv[kMergeGroup];
+#pragma unroll
+    for (int g = 0; g < kMergeGroup; ++g) {
+      const bool on = i0 + g < n_split;
+      const float* si = row0 + static_cast<size_t>(i0 + g) * slot_elems;
+      mv[g] = on ? __ldcg(si + static_cast<size_t>(d) * kRows) : -INFINITY;
+      lv[g] = on ? __ldcg(si + static_cast<size_t>(d + 1) * kRows) : 0.f;
+    }
+    float mn = mr;
+#pragma unroll
+    for (int g = 0; g < kMergeGroup; ++g) mn = fmaxf(mn, mv[g]);
+    ls *= ex2(mr - mn);  // 0 on the first group (mr = -inf); every part's m is finite
+#pragma unroll
+    for (int g = 0; g < kMergeGroup; ++g) ls += ex2(mv[g] - mn) * lv[g];  // absent parts add 0
+    mr = mn;
+  }
+  mref = mr;
+  inv = 1.f / ls;
+}
+
+// Columns c_begin .. c_begin + NCOLS - 1 of the merged row, in blocks of CB columns, to bf16
+// at dst (which points at column c_begin of the output row).  NCOLS and CB are multiples of 8.
+template <int NCOLS, int CB>
+__device__ __forceinline__ void merge_columns(const float* row0, size_t slot_elems, int d, int n_split,
+                                              int c_begin, float mref, float inv, uint16_t* dst,
+                                              bool in_range) {
+  static_assert(NCOLS % 8 == 0 && CB % 8 == 0, "whole 16-byte stores");
+#pragma unroll
+  for (int cb = 0; cb < NCOLS; cb += CB) {
+    constexpr int kFull = CB;
+    const int nc = NCOLS - cb < kFull ? NCOLS - cb : kFull;  // constant once unrolled
+    float acc[CB];
+#pragma unroll
+    for (int k = 0; k < CB; ++k) acc[k] = 0.f;
+    for (int i0 = 0; i0 < n_split; i0 += kMergeGroup) {
+      float v[kMergeGroup][CB], mv[kMergeGroup];
+#pragma unroll
+      for (int g = 0; g < kMergeGroup; ++g) {
+        const bool on = i0 + g < n_split;
+        const float* si = row0 + static_cast<size_t>(i0 + g) * slot_elems;
+        mv[g] = on ? __ldcg(si + static_cast<size_t>(d) * kRows) : -INFINITY;
+#pragma unroll
+        for (int k = 0; k < CB; ++k)
+          if (k < nc) v[g][k] = on ? __ldcg(si + static_cast<size_t>(c_begin + cb + k) * kRows) : 0.f;
+      }
+#pragma unroll
+      for (int g = 0; g < kMergeGroup; ++g) {
+        const float w = ex2(mv[g] - mref) * inv;
+#pragma unroll
+        for (int k = 0; k < CB; ++k)
+          if (k < nc) acc[k] = fmaf(w, v[g][k], acc[k]);
+      }
+    }
+    if (in_range) {
+#pragma unroll
+      for (int k = 0; k < CB; k += 8) {
+        if (k < nc) {
+          uint4 w0;
+          w0.x = pack_bf16(acc[k + 0], acc[k + 1]);
+          w0.y = pack_bf16(acc[k + 2], acc[k + 3]);
+          w0.z = pack_bf16(acc[k + 4], acc[k + 5]);
+          w0.w = pack_bf16(acc[k + 6], acc[k + 7]);
+          *reinterpret_cast<uint4*>(dst + cb + k) = w0;
+        }
+      }
+    }
+  }
+}
+
 // Barrier among the `count` threads of one softmax warpgroup (ids 1 and 2; 0 is __syncthreads).
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -287,6 +380,29 @@ __device__ __forceinline__ void scatter_share(const AttnParams& p, int lane) {
 // After the merge, the partial slots of a query tile ([part][d + 2][128] fp32) are dead: the next launch writes every slot before it reads one.  Dropping their L2 lines
 // keeps them from being written back to DRAM.  `tid` / `nthreads` split the lines among the
 // merging threads.
+// Which (pair, part) a CTA computes.  CTAs are numbered (batch x head, part, query-tile
+// group): the query-tile groups of one head that read the same key range are neighbours, so
+// they run in the same wave and read each context tile from DRAM about once while it sits in
+// L2; where a wave ends inside a head, only the key range of one part is read twice (the
+// waves of a launch rarely hold whole heads).  The parts of a pair are n_groups CTAs apart,
+// within one wave for all but the CTAs at a wave's end, so the last part usually merges
+// partials that are still in L2.
+struct CtaWork {
+  int pair, part, grp, hd, b;
+};
+__device__ __forceinline__ CtaWork cta_work(const AttnParams& p) {
+  const int per_bh = p.n_groups * p.n_split;
+  const int bh = static_cast<int>(blockIdx.x) / per_bh;
+  const int rem = static_cast<int>(blockIdx.x) - bh * per_bh;
+  CtaWork w;
+  w.part = rem / p.n_groups;
+  w.grp = rem - w.part * p.n_groups;
+  w.pair = bh * p.n_groups + w.grp;
+  w.hd = bh % p.heads;
+  w.b = bh / p.heads;
+  return w;
+}
+
 template <int D>
 __device__ __forceinline__ void discard_partials(const float* slot0, int n_split, int tid, int nthreads) {
   static_assert((D + 2) * kRows * 4 % 128 == 0, "slots are whole 128-byte lines");
@@ -406,14 +522,9 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
   PF_TRACE_CTA(1);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // pair-major order: the parts of one query-tile pair run in the same wave, so the partials
-  // they write are merged while still in L2, and a wave's CTAs share few heads' context
-  const int pair = blockIdx.x / p.n_split;
-  const int part = blockIdx.x - pair * p.n_split;
-  const int grp = pair % p.n_groups;
-  const int hd = (pair / p.n_groups) % p.heads;
-  const int b = pair / (p.n_groups * p.heads);
-  const int q0 = grp * NQ * kRows;
+  const CtaWork wk = cta_work(p);
+  const int pair = wk.pair, part = wk.part, hd = wk.hd, b = wk.b;
+  const int q0 = wk.grp * NQ * kRows;
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
@@ -460,6 +571,7 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  PF_TRACE_EV(0);
   // the next micro-step may start its CTAs (set-up, Q and fresh K/V loads) on SMs this grid
   // leaves idle; everything that touches memory this grid writes waits (grid_dep_wait)
   grid_dep_launch();
@@ -617,6 +729,7 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
       if (!s_ready) ok = ok && mbar_wait(smem_u32(s_full + t), j & 1, abort, kWaitNs);
       tc_fence_after();
       if (wq == 0 && lane == 0) PF_TRACE_AT(0, 2 * t + hh, j);
+      if (j == 0) PF_TRACE_EV(1);
       uint32_t s[64];
       tmem_ld32(tS + 0, s);
       tmem_ld32(tS + 32, s + 32);
@@ -715,6 +828,7 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
     if (!ok && lane == 0) raise_abort(abort, kWdSoftmax);
     {
       bool ok_o = ok && mbar_wait(smem_u32(o_full + t), 0, abort, kWaitNs);
+      PF_TRACE_EV(2);
       ok_o = __all_sync(0xffffffffu, ok_o);
       // both halves of the query tile take the same branch (the epilogue has barriers)
       ok_o = named_bar_and(9 + t, 2 * kRows, ok_o);
@@ -766,6 +880,7 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
           }
           __threadfence();
           named_bar_sync(9 + t, 2 * kRows);
+          PF_TRACE_EV(3);
           if (hh == 0 && rloc == 0) {
             const unsigned old = atomicAdd(p.ws_cnt + pair * 2 + t, 1u);
             const int last = old == static_cast<unsigned>(p.n_split - 1);
@@ -776,43 +891,16 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
             s_last[t] = last;
           }
           named_bar_sync(9 + t, 2 * kRows);
+          PF_TRACE_EV(4);
           if (s_last[t]) {
             // merge every part of this query tile: this thread's 32 columns of its row
-            float mref = -INFINITY, lsum = 0.f;
-#pragma unroll 4
-            for (int i = 0; i < p.n_split; ++i)
-              mref = fmaxf(mref, __ldcg(slot0 + i * slot_elems + D * kRows + rloc));
-#pragma unroll 4
-            for (int i = 0; i < p.n_split; ++i) {
-              const float* si = slot0 + i * slot_elems;
-              lsum += ex2(__ldcg(si + D * kRows + rloc) - mref) * __ldcg(si + (D + 1) * kRows + rloc);
-            }
-            const float inv = 1.f / lsum;
-            float acc[32];
-#pragma unroll
-            for (int k = 0; k < 32; ++k) acc[k] = 0.f;
-            for (int i = 0; i < p.n_split; ++i) {
-              const float* si = slot0 + i * slot_elems + rloc;
-              float v[32];
-#pragma unroll
-              for (int k = 0; k < 32; ++k) v[k] = __ldcg(si + (32 * hh + k) * kRows);
-              const float w = ex2(__ldcg(si + D * kRows) - mref) * inv;
-#pragma unroll
-              for (int k = 0; k < 32; ++k) acc[k] = fmaf(w, v[k], acc[k]);
-            }
-            if (in_range) {
-#pragma unroll
-              for (int k = 0; k < 32; k += 8) {
-                uint4 w;
-                w.x = pack_bf16(acc[k + 0], acc[k + 1]);
-                w.y = pack_bf16(acc[k + 2], acc[k + 3]);
-                w.z = pack_bf16(acc[k + 4], acc[k + 5]);
-                w.w = pack_bf16(acc[k + 6], acc[k + 7]);
-                *reinterpret_cast<uint4*>(dst + k) = w;
-              }
-            }
+            float mref, inv;
+            merge_stats(slot0 + rloc, slot_elems, D, p.n_split, mref, inv);
+            merge_columns<32, 16>(slot0 + rloc, slot_elems, D, p.n_split, 32 * hh, mref, inv, dst,
+                                 in_range);
             // every thread of the tile has read all parts' slots: drop them from L2
             named_bar_sync(9 + t, 2 * kRows);
+            PF_TRACE_EV(5);
             discard_partials<D>(slot0, p.n_split, hh * kRows + rloc, 2 * kRows);
           }
         }
@@ -927,6 +1015,7 @@ __device__ __forceinline__ void full_row_epilogue(const AttnParams& p, uint32_t 
   mine[(D + 1) * kRows + rloc] = l;
   __threadfence();
   named_bar_sync(1 + t, kRows);
+  PF_TRACE_EV(3);
   if (rloc == 0) {
     const unsigned old = atomicAdd(p.ws_cnt + pair * 2 + t, 1u);
     const int last = old == static_cast<unsigned>(p.n_split - 1);
@@ -937,53 +1026,15 @@ __device__ __forceinline__ void full_row_epilogue(const AttnParams& p, uint32_t 
     s_last[t] = last;
   }
   named_bar_sync(1 + t, kRows);
+  PF_TRACE_EV(4);
   if (!s_last[t]) return;
-  // Merge every part of this query tile.  Each round trip to L2 fetches a whole 64-column
-  // block of one part's row (or every part's m and l).
-  float mref = -INFINITY, lsum = 0.f;
-#pragma unroll 4
-  for (int i = 0; i < p.n_split; ++i)
-    mref = fmaxf(mref, __ldcg(slot0 + i * slot_elems + D * kRows + rloc));
-#pragma unroll 4
-  for (int i = 0; i < p.n_split; ++i) {
-    const float* si = slot0 + i * slot_elems;
-    lsum += ex2(__ldcg(si + D * kRows + rloc) - mref) * __ldcg(si + (D + 1) * kRows + rloc);
-  }
-  const float inv = 1.f / lsum;
-#pragma unroll
-  for (int cb = 0; cb < D; cb += 64) {
-    constexpr int kBlock = 64;
-    const int nc = D - cb < kBlock ? D - cb : kBlock;  // constant once unrolled
-    float acc[kBlock];
-#pragma unroll
-    for (int k = 0; k < kBlock; ++k) acc[k] = 0.f;
-    for (int i = 0; i < p.n_split; ++i) {
-      const float* si = slot0 + i * slot_elems + rloc;
-      float v[kBlock];
-#pragma unroll
-      for (int k = 0; k < kBlock; ++k)
-        if (k < nc) v[k] = __ldcg(si + (cb + k) * kRows);
-      const float w = ex2(__ldcg(si + D * kRows) - mref) * inv;
-#pragma unroll
-      for (int k = 0; k < kBlock; ++k)
-        if (k < nc) acc[k] = fmaf(w, v[k], acc[k]);
-    }
-    if (in_range) {
-#pragma unroll
-      for (int k = 0; k < kBlock; k += 8) {
-        if (k < nc) {
-          uint4 w0;
-          w0.x = pack_bf16(acc[k + 0], acc[k + 1]);
-          w0.y = pack_bf16(acc[k + 2], acc[k + 3]);
-          w0.z = pack_bf16(acc[k + 4], acc[k + 5]);
-          w0.w = pack_bf16(acc[k + 6], acc[k + 7]);
-          *reinterpret_cast<uint4*>(dst + cb + k) = w0;
-        }
-      }
-    }
-  }
+  // merge every part of this query tile
+  float mref, inv;
+  merge_stats(slot0 + rloc, slot_elems, D, p.n_split, mref, inv);
+  merge_columns<D, 24>(slot0 + rloc, slot_elems, D, p.n_split, 0, mref, inv, dst, in_range);
   // every thread of the tile has read all parts' slots: drop them from L2
   named_bar_sync(1 + t, kRows);
+  PF_TRACE_EV(5);
   discard_partials<D>(slot0, p.n_split, rloc, kRows);
 }
 
@@ -1031,14 +1082,9 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
   PF_TRACE_CTA(1);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // pair-major order: the parts of one query-tile pair run in the same wave, so the partials
-  // they write are merged while still in L2, and a wave's CTAs share few heads' context
-  const int pair = blockIdx.x / p.n_split;
-  const int part = blockIdx.x - pair * p.n_split;
-  const int grp = pair % p.n_groups;
-  const int hd = (pair / p.n_groups) % p.heads;
-  const int b = pair / (p.n_groups * p.heads);
-  const int q0 = grp * NQ * kRows;
+  const CtaWork wk = cta_work(p);
+  const int pair = wk.pair, part = wk.part, hd = wk.hd, b = wk.b;
+  const int q0 = wk.grp * NQ * kRows;
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
@@ -1086,6 +1132,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  PF_TRACE_EV(0);
   // the next micro-step may start its CTAs (set-up, Q and fresh K/V loads) on SMs this grid
   // leaves idle; everything that touches memory this grid writes waits (grid_dep_wait)
   grid_dep_launch();
@@ -1257,6 +1304,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
         if (!ok) break;
         tc_fence_after();
         if (wq == 0 && lane == 0) PF_TRACE_AT(0, 2 * t + h, j);
+        if (j == 0 && h == 0) PF_TRACE_EV(1);
         uint32_t s[64];
         tmem_ld32(tS + h * 64, s);
         tmem_ld32(tS + h * 64 + 32, s + 32);
@@ -1313,6 +1361,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
     if (!ok && lane == 0) raise_abort(abort, kWdSoftmax);
     {
       bool ok_o = ok && mbar_wait(smem_u32(o_full + t), 0, abort, kWaitNs);
+      PF_TRACE_EV(2);
       ok_o = __all_sync(0xffffffffu, ok_o);
       // the whole warpgroup takes the same branch (the merge path has barriers)
       ok_o = named_bar_and(1 + t, kRows, ok_o);
@@ -1436,6 +1485,10 @@ extern "C" int pf_trace_read(unsigned long long* dst, size_t n) {
 extern "C" int pf_trace_cta_read(unsigned long long* dst, size_t n) {
   if (n > sizeof(g_cta) / sizeof(g_cta[0])) n = sizeof(g_cta) / sizeof(g_cta[0]);
   return static_cast<int>(cudaMemcpyFromSymbol(dst, g_cta, n * sizeof(unsigned long long)));
+}
+extern "C" int pf_trace_ev_read(unsigned long long* dst, size_t n) {
+  if (n > sizeof(g_cta_ev) / sizeof(g_cta_ev[0])) n = sizeof(g_cta_ev) / sizeof(g_cta_ev[0]);
+  return static_cast<int>(cudaMemcpyFromSymbol(dst, g_cta_ev, n * sizeof(unsigned long long)));
 }
 #endif
 
