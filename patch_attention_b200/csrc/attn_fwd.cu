@@ -202,23 +202,24 @@ __device__ __forceinline__ void store_row16(uint16_t* dst, int c0, const uint32_
   }
 }
 
-// Merging the key-range parts of one query row.  Part i's slot holds, column-major with
-// kRows rows per column, the unnormalised O row (d columns) and then m_i and l_i; row0
-// points at this row's entry of part 0's slot.  The merged row is
+// Merging the key-range parts of one query row.  The merger is the last part to finish its
+// loop; its own part stays in registers (m, l) and TMEM (O).  Every other part i has stored,
+// column-major with kRows rows per column, its unnormalised O row (d columns) and then m_i
+// and l_i in its slot; row0 points at this row's entry of part 0's slot.  The merged row is
 //   O = sum_i 2^(m_i - mref) O_i / sum_i 2^(m_i - mref) l_i,   mref = max_i m_i
 // (log-sum-exp combination of softmax parts).  The slots sit in L2, written by other CTAs,
 // so the merge is bound by L2 round trips: loads are issued for four parts at a time (and
-// for the O row, a block of columns of all four) before any of them is used.
+// for the O row, 16 columns of all four) before any of them is used.
 constexpr int kMergeGroup = 4;
 
 __device__ __forceinline__ void merge_stats(const float* row0, size_t slot_elems, int d, int n_split,
-                                            float& mref, float& inv) {
-  float mr = -INFINITY, ls = 0.f;
+                                            int own, float m_own, float l_own, float& mref, float& inv) {
+  float mr = m_own, ls = l_own;
   for (int i0 = 0; i0 < n_split; i0 += kMergeGroup) {
     float mv[kMergeGroup], lv[kMergeGroup];
 #pragma unroll
     for (int g = 0; g < kMergeGroup; ++g) {
-      const bool on = i0 + g < n_split;
+      const bool on = i0 + g < n_split && i0 + g != own;
       const float* si = row0 + static_cast<size_t>(i0 + g) * slot_elems;
       mv[g] = on ? __ldcg(si + static_cast<size_t>(d) * kRows) : -INFINITY;
       lv[g] = on ? __ldcg(si + static_cast<size_t>(d + 1) * kRows) : 0.f;
@@ -226,7 +227,7 @@ __device__ __forceinline__ void merge_stats(const float* row0, size_t slot_elems
     float mn = mr;
 #pragma unroll
     for (int g = 0; g < kMergeGroup; ++g) mn = fmaxf(mn, mv[g]);
-    ls *= ex2(mr - mn);  // 0 on the first group (mr = -inf); every part's m is finite
+    ls *= ex2(mr - mn);  // every part's m is finite
 #pragma unroll
     for (int g = 0; g < kMergeGroup; ++g) ls += ex2(mv[g] - mn) * lv[g];  // absent parts add 0
     mr = mn;
@@ -235,25 +236,31 @@ __device__ __forceinline__ void merge_stats(const float* row0, size_t slot_elems
   inv = 1.f / ls;
 }
 
-// Columns c_begin .. c_begin + NCOLS - 1 of the merged row, in blocks of CB columns, to bf16
-// at dst (which points at column c_begin of the output row).  NCOLS and CB are multiples of 8.
-template <int NCOLS, int CB>
+// Columns c_begin .. c_begin + NCOLS - 1 of the merged row to bf16 at dst (which points at
+// column c_begin of the output row), 16 at a time; tO is the TMEM address of the merger's own
+// O at column c_begin (this thread's lane), w_own its weight 2^(m_own - mref) / sum.  Warp-
+// collective (TMEM loads).  NCOLS is a multiple of 8; TMEM holds O padded to 16 columns.
+template <int NCOLS>
 __device__ __forceinline__ void merge_columns(const float* row0, size_t slot_elems, int d, int n_split,
-                                              int c_begin, float mref, float inv, uint16_t* dst,
-                                              bool in_range) {
-  static_assert(NCOLS % 8 == 0 && CB % 8 == 0, "whole 16-byte stores");
+                                              int own, int c_begin, uint32_t tO, float w_own,
+                                              float mref, float inv, uint16_t* dst, bool in_range) {
+  static_assert(NCOLS % 8 == 0, "whole 16-byte stores");
+  constexpr int CB = 16;
 #pragma unroll
   for (int cb = 0; cb < NCOLS; cb += CB) {
-    constexpr int kFull = CB;
-    const int nc = NCOLS - cb < kFull ? NCOLS - cb : kFull;  // constant once unrolled
+    const int nc = NCOLS - cb < CB ? NCOLS - cb : CB;  // constant once unrolled
+    uint32_t o[CB];
+    tmem_ld16(tO + static_cast<uint32_t>(cb), o);
+    tmem_wait_ld();
+    reg_fence<CB>(o);
     float acc[CB];
 #pragma unroll
-    for (int k = 0; k < CB; ++k) acc[k] = 0.f;
+    for (int k = 0; k < CB; ++k) acc[k] = w_own * __uint_as_float(o[k]);
     for (int i0 = 0; i0 < n_split; i0 += kMergeGroup) {
       float v[kMergeGroup][CB], mv[kMergeGroup];
 #pragma unroll
       for (int g = 0; g < kMergeGroup; ++g) {
-        const bool on = i0 + g < n_split;
+        const bool on = i0 + g < n_split && i0 + g != own;
         const float* si = row0 + static_cast<size_t>(i0 + g) * slot_elems;
         mv[g] = on ? __ldcg(si + static_cast<size_t>(d) * kRows) : -INFINITY;
 #pragma unroll
@@ -403,14 +410,22 @@ __device__ __forceinline__ CtaWork cta_work(const AttnParams& p) {
   return w;
 }
 
+// After a merge: mark the other parts' slots of the query tile dead in L2 (the merger's own
+// slot was never written), so they are dropped instead of written back to DRAM.
 template <int D>
-__device__ __forceinline__ void discard_partials(const float* slot0, int n_split, int tid, int nthreads) {
+__device__ __forceinline__ void discard_partials(const float* slot0, int n_split, int own, int tid,
+                                                 int nthreads) {
   static_assert((D + 2) * kRows * 4 % 128 == 0, "slots are whole 128-byte lines");
+  constexpr int kLines = (D + 2) * kRows * 4 / 128;  // per slot
   const char* base = reinterpret_cast<const char*>(slot0);
   // the workspace only has to be 16-byte aligned: skip when the lines are not whole
   if ((reinterpret_cast<uintptr_t>(base) & 127u) != 0) return;
-  const int lines = n_split * (D + 2) * kRows * 4 / 128;
-  for (int i = tid; i < lines; i += nthreads) discard_l2_line(base + static_cast<size_t>(i) * 128);
+  const int lines = (n_split - 1) * kLines;
+  for (int i = tid; i < lines; i += nthreads) {
+    const int slot = i / kLines;
+    const int idx = (slot >= own ? slot + 1 : slot) * kLines + (i - slot * kLines);
+    discard_l2_line(base + static_cast<size_t>(idx) * 128);
+  }
 }
 
 // ------------------------------------------------------------------ head_dim 64: half rows
@@ -517,7 +532,7 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   __shared__ float xch_m[2][2][2][kRows];  // [tile parity][t][half][row]: half-tile maxima
   __shared__ float xch_l[2][2][kRows];     // [t][half][row]: row sums at the end
-  __shared__ int s_last[2];
+  __shared__ int s_last[4];  // [t]: this CTA merges query tile t; [2 + t]: the partials are ready
 
   PF_TRACE_CTA(1);
   const int warp = threadIdx.x >> 5;
@@ -868,40 +883,55 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
             }
           }
         } else {
-          // partial: O row (64 columns, this thread's 32), m, l into this part's slot, column-major
+          // the last part to finish its loop merges (an arrival counter tells, before anything
+          // is stored); the others store their partial and count it written
           const size_t slot_elems = static_cast<size_t>(D + 2) * kRows;
           float* slot0 = p.ws_part + (static_cast<size_t>(pair) * 2 + t) * p.n_split * slot_elems;
-          float* mine = slot0 + static_cast<size_t>(part) * slot_elems;
+          unsigned* cnt = p.ws_cnt + (static_cast<size_t>(pair) * 2 + t) * 2;  // arrived, written
+          if (hh == 0 && rloc == 0) s_last[t] = atomicAdd(cnt, 1u) == static_cast<unsigned>(p.n_split - 1);
+          named_bar_sync(9 + t, 2 * kRows);
+          if (!s_last[t]) {
+            // partial: O row (64 columns, this thread's 32), m, l into this part's slot, column-major
+            float* mine = slot0 + static_cast<size_t>(part) * slot_elems;
 #pragma unroll
-          for (int k = 0; k < 32; ++k) mine[(32 * hh + k) * kRows + rloc] = o[k];
-          if (hh == 0) {
-            mine[D * kRows + rloc] = m;
-            mine[(D + 1) * kRows + rloc] = lrow;
-          }
-          __threadfence();
-          named_bar_sync(9 + t, 2 * kRows);
-          PF_TRACE_EV(3);
-          if (hh == 0 && rloc == 0) {
-            const unsigned old = atomicAdd(p.ws_cnt + pair * 2 + t, 1u);
-            const int last = old == static_cast<unsigned>(p.n_split - 1);
-            if (last) {
-              __threadfence();
-              p.ws_cnt[pair * 2 + t] = 0u;  // ready for the next launch
+            for (int k = 0; k < 32; ++k) mine[(32 * hh + k) * kRows + rloc] = o[k];
+            if (hh == 0) {
+              mine[D * kRows + rloc] = m;
+              mine[(D + 1) * kRows + rloc] = lrow;
             }
-            s_last[t] = last;
-          }
-          named_bar_sync(9 + t, 2 * kRows);
-          PF_TRACE_EV(4);
-          if (s_last[t]) {
-            // merge every part of this query tile: this thread's 32 columns of its row
-            float mref, inv;
-            merge_stats(slot0 + rloc, slot_elems, D, p.n_split, mref, inv);
-            merge_columns<32, 16>(slot0 + rloc, slot_elems, D, p.n_split, 32 * hh, mref, inv, dst,
-                                 in_range);
-            // every thread of the tile has read all parts' slots: drop them from L2
+            __threadfence();
             named_bar_sync(9 + t, 2 * kRows);
-            PF_TRACE_EV(5);
-            discard_partials<D>(slot0, p.n_split, hh * kRows + rloc, 2 * kRows);
+            PF_TRACE_EV(3);
+            if (hh == 0 && rloc == 0) atomicAdd(cnt + 1, 1u);
+          } else {
+            // the merger: wait (bounded) for the other parts' partials -- they have all arrived,
+            // so they are running and wait for nothing -- then reset the counters for the next
+            // launch and combine them with its own part, which it never stores
+            if (hh == 0 && rloc == 0) {
+              const bool ready = wait_count_geq(cnt + 1, static_cast<unsigned>(p.n_split - 1), abort, kWaitNs);
+              if (ready) {
+                cnt[0] = 0u;
+                cnt[1] = 0u;
+              } else {
+                raise_abort(abort, kWdEpilogue);
+              }
+              s_last[2 + t] = ready;
+            }
+            named_bar_sync(9 + t, 2 * kRows);
+            PF_TRACE_EV(4);
+            if (s_last[2 + t]) {
+              // this thread's 32 columns of its row
+              float mref, inv;
+              merge_stats(slot0 + rloc, slot_elems, D, p.n_split, part, m, lrow, mref, inv);
+              merge_columns<32>(slot0 + rloc, slot_elems, D, p.n_split, part, 32 * hh, tO,
+                                ex2(m - mref) * inv, mref, inv, dst, in_range);
+              PF_TRACE_EV(5);
+              if (p.discard) {
+                // every thread of the tile has read the other parts' slots: drop them from L2
+                named_bar_sync(9 + t, 2 * kRows);
+                discard_partials<D>(slot0, p.n_split, part, hh * kRows + rloc, 2 * kRows);
+              }
+            }
           }
         }
       }
@@ -972,14 +1002,17 @@ cudaError_t launch_hr(const AttnParams& p, cudaStream_t stream) {
 }
 
 // Epilogue of a softmax thread that owns a whole query row: O (TMEM columns from tO) over l
-// to the bf16 output when the call has no key-range split; otherwise the unnormalised row
-// with its m and l goes to this part's workspace slot, and the last part of the query tile
-// to finish (an atomic counter decides) merges all parts.  Called by all 128 threads of the
-// query tile's warpgroup (named barrier 1 + t).
+// to the bf16 output when the call has no key-range split.  Otherwise the last part of the
+// query tile to finish its loop (an arrival counter tells, before anything is stored) merges:
+// every other part stores its unnormalised row with m and l in its workspace slot and counts
+// it written; the merger waits (bounded) for those counts -- the parts it waits for have all
+// arrived, so they are running and wait for nothing -- and combines them with its own part,
+// which it never stores.  Called by all 128 threads of the query tile's warpgroup (named
+// barrier 1 + t).
 template <int D>
 __device__ __forceinline__ void full_row_epilogue(const AttnParams& p, uint32_t tO, float m, float l,
                                                   int pair, int part, int t, int q0, int hd, int b,
-                                                  int wq, int lane, int* s_last) {
+                                                  int wq, int lane, int* s_last, volatile int* abort) {
   constexpr int kMmaN = Dims<D>::kMmaN;
   const int rloc = wq * 32 + lane;
   const int row = q0 + t * kRows + rloc;
@@ -997,45 +1030,54 @@ __device__ __forceinline__ void full_row_epilogue(const AttnParams& p, uint32_t 
     }
     return;
   }
-  // partial: O row (d columns), m, l into this part's slot, column-major
   const size_t slot_elems = static_cast<size_t>(D + 2) * kRows;
   float* slot0 = p.ws_part + (static_cast<size_t>(pair) * 2 + t) * p.n_split * slot_elems;
-  float* mine = slot0 + static_cast<size_t>(part) * slot_elems;
-#pragma unroll
-  for (int c0 = 0; c0 < kMmaN; c0 += 16) {
-    uint32_t o[16];
-    tmem_ld16(tO + c0, o);
-    tmem_wait_ld();
-    reg_fence<16>(o);
-#pragma unroll
-    for (int k = 0; k < 16; ++k)
-      if (c0 + k < D) mine[(c0 + k) * kRows + rloc] = __uint_as_float(o[k]);
-  }
-  mine[D * kRows + rloc] = m;
-  mine[(D + 1) * kRows + rloc] = l;
-  __threadfence();
+  unsigned* cnt = p.ws_cnt + (static_cast<size_t>(pair) * 2 + t) * 2;  // arrived, written
+  if (rloc == 0) s_last[t] = atomicAdd(cnt, 1u) == static_cast<unsigned>(p.n_split - 1);
   named_bar_sync(1 + t, kRows);
-  PF_TRACE_EV(3);
-  if (rloc == 0) {
-    const unsigned old = atomicAdd(p.ws_cnt + pair * 2 + t, 1u);
-    const int last = old == static_cast<unsigned>(p.n_split - 1);
-    if (last) {
-      __threadfence();
-      p.ws_cnt[pair * 2 + t] = 0u;  // ready for the next launch
+  if (!s_last[t]) {
+    // partial: O row (d columns), m, l into this part's slot, column-major
+    float* mine = slot0 + static_cast<size_t>(part) * slot_elems;
+#pragma unroll
+    for (int c0 = 0; c0 < kMmaN; c0 += 16) {
+      uint32_t o[16];
+      tmem_ld16(tO + c0, o);
+      tmem_wait_ld();
+      reg_fence<16>(o);
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        if (c0 + k < D) mine[(c0 + k) * kRows + rloc] = __uint_as_float(o[k]);
     }
-    s_last[t] = last;
+    mine[D * kRows + rloc] = m;
+    mine[(D + 1) * kRows + rloc] = l;
+    __threadfence();
+    named_bar_sync(1 + t, kRows);
+    if (rloc == 0) atomicAdd(cnt + 1, 1u);
+    return;
+  }
+  // the merger: wait until the other parts' partials are written, then reset the counters
+  // for the next launch (every other part has counted both by then)
+  if (rloc == 0) {
+    const bool ready = wait_count_geq(cnt + 1, static_cast<unsigned>(p.n_split - 1), abort, kWaitNs);
+    if (ready) {
+      cnt[0] = 0u;
+      cnt[1] = 0u;
+    } else {
+      raise_abort(abort, kWdEpilogue);
+    }
+    s_last[2 + t] = ready;
   }
   named_bar_sync(1 + t, kRows);
-  PF_TRACE_EV(4);
-  if (!s_last[t]) return;
-  // merge every part of this query tile
+  if (!s_last[2 + t]) return;
   float mref, inv;
-  merge_stats(slot0 + rloc, slot_elems, D, p.n_split, mref, inv);
-  merge_columns<D, 24>(slot0 + rloc, slot_elems, D, p.n_split, 0, mref, inv, dst, in_range);
-  // every thread of the tile has read all parts' slots: drop them from L2
-  named_bar_sync(1 + t, kRows);
-  PF_TRACE_EV(5);
-  discard_partials<D>(slot0, p.n_split, rloc, kRows);
+  merge_stats(slot0 + rloc, slot_elems, D, p.n_split, part, m, l, mref, inv);
+  merge_columns<D>(slot0 + rloc, slot_elems, D, p.n_split, part, 0, tO, ex2(m - mref) * inv, mref, inv,
+                   dst, in_range);
+  if (p.discard) {
+    // every thread of the tile has read the other parts' slots: drop them from L2
+    named_bar_sync(1 + t, kRows);
+    discard_partials<D>(slot0, p.n_split, part, rloc, kRows);
+  }
 }
 
 // ------------------------------------------------------------------ head_dim 72/128: split key tiles
@@ -1077,7 +1119,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
   uint64_t* mma_done = o_full + 2;   // [issuer]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  __shared__ int s_last[2];
+  __shared__ int s_last[4];  // [t]: this CTA merges query tile t; [2 + t]: the partials are ready
 
   PF_TRACE_CTA(1);
   const int warp = threadIdx.x >> 5;
@@ -1370,7 +1412,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
       } else {
         tc_fence_after();
         grid_dep_wait();  // the output and the workspace may be in use by the previous grid
-        full_row_epilogue<D>(p, tO, m, l, pair, part, t, q0, hd, b, wq, lane, s_last);
+        full_row_epilogue<D>(p, tO, m, l, pair, part, t, q0, hd, b, wq, lane, s_last, abort);
       }
     }
   } else {
@@ -1455,7 +1497,7 @@ int attn_choose_split(int n_pairs, int n_tiles, int n_sms, int max_split) {
 size_t attn_workspace_bytes(int n_pairs, int head_dim, int n_split) {
   if (n_split <= 1) return 0;
   const size_t part_bytes = static_cast<size_t>(n_pairs) * 2 * n_split * (head_dim + 2) * kRows * 4;
-  const size_t cnt_bytes = static_cast<size_t>(n_pairs) * 2 * 4;
+  const size_t cnt_bytes = static_cast<size_t>(n_pairs) * 2 * 2 * 4;
   return ((part_bytes + 255) / 256) * 256 + cnt_bytes;
 }
 

@@ -122,7 +122,8 @@ constexpr int kAssumedSms = 148;
 
 // Counters first (fixed place, sized for the larger of patch and text-query calls), then the
 // partial slots.
-size_t counter_bytes(int pairs) { return ((static_cast<size_t>(pairs) * 2 * 4 + 255) / 256) * 256; }
+// Two counters (parts arrived, partials written) per query tile of every pair.
+size_t counter_bytes(int pairs) { return ((static_cast<size_t>(pairs) * 2 * 2 * 4 + 255) / 256) * 256; }
 
 size_t workspace_for(const pf_config& c, int n_sms) {
   const int plen = c.n_img / c.n_patches;
@@ -176,6 +177,10 @@ cudaError_t launch_attention(pf_ctx* ctx, pf::AttnParams& p, void* stream) {
     if (p.n_split > 1) {
       p.ws_cnt = reinterpret_cast<unsigned*>(ctx->ws);
       p.ws_part = reinterpret_cast<float*>(ctx->ws + cb);
+      // a launch of several waves keeps writing partials while earlier ones are merged: drop
+      // the merged ones from L2 instead of letting them go back to DRAM; a single wave's few
+      // partials cost less to write back than the discard costs at the end of the launch
+      p.discard = static_cast<long long>(p.n_pairs) * p.n_split > ctx->n_sms ? 1 : 0;
     }
   }
   return pf::launch_patch_attn(p, static_cast<cudaStream_t>(stream));

@@ -41,7 +41,8 @@ struct AttnParams {
   int n_pairs;          // batch * heads * n_groups
   int n_split;          // parts per pair (1 => no partials)
   float* ws_part;       // partial (O, m, l) slots, [pair][tile][part][d + 2][128] fp32
-  unsigned* ws_cnt;     // finished-part counters, [pair][tile]; zero between launches
+  unsigned* ws_cnt;     // per [pair][tile]: parts arrived, partials written; zero between launches
+  int discard;          // drop the merged partials from L2 (1) rather than let them be written back
 };
 
 // Query tiles per CTA chosen for a patch length (1 or 2).

@@ -101,6 +101,22 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// Wait until the 32-bit counter at c (global memory, written by other CTAs) reaches target:
+// acquire loads with a short sleep between them, bounded by limit_ns (false when it gave up)
+// and by the abort flag.
+__device__ __forceinline__ bool wait_count_geq(const unsigned* c, unsigned target,
+                                               const volatile int* abort, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
+    if (v >= target) return true;
+    if (abort != nullptr && *abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+    __nanosleep(100);
+  }
+}
+
 // ------------------------------------------------------------------ programmatic dependent launch
 
 // Let the next grid on the stream (launched with programmatic stream serialization) start
