@@ -202,24 +202,24 @@ __device__ __forceinline__ void store_row16(uint16_t* dst, int c0, const uint32_
   }
 }
 
-// Merging the key-range parts of one query row.  The merger is the last part to finish its
-// loop; its own part stays in registers (m, l) and TMEM (O).  Every other part i has stored,
-// column-major with kRows rows per column, its unnormalised O row (d columns) and then m_i
-// and l_i in its slot; row0 points at this row's entry of part 0's slot.  The merged row is
+// Merging the key-range parts of one query row.  Part i's slot holds, column-major with
+// kRows rows per column, the unnormalised O row (d columns) and then m_i and l_i; row0
+// points at this row's entry of part 0's slot.  The merged row is
 //   O = sum_i 2^(m_i - mref) O_i / sum_i 2^(m_i - mref) l_i,   mref = max_i m_i
-// (log-sum-exp combination of softmax parts).  The slots sit in L2, written by other CTAs,
-// so the merge is bound by L2 round trips: loads are issued for four parts at a time (and
-// for the O row, 16 columns of all four) before any of them is used.
+// (log-sum-exp combination of softmax parts), summed in part order whichever part merges.
+// The slots sit in L2, written by other CTAs, so the merge is bound by L2 round trips: loads
+// are issued for four parts at a time (and for the O row, 16 columns of all four) before any
+// of them is used.
 constexpr int kMergeGroup = 4;
 
 __device__ __forceinline__ void merge_stats(const float* row0, size_t slot_elems, int d, int n_split,
-                                            int own, float m_own, float l_own, float& mref, float& inv) {
-  float mr = m_own, ls = l_own;
+                                            float& mref, float& inv) {
+  float mr = -INFINITY, ls = 0.f;
   for (int i0 = 0; i0 < n_split; i0 += kMergeGroup) {
     float mv[kMergeGroup], lv[kMergeGroup];
 #pragma unroll
     for (int g = 0; g < kMergeGroup; ++g) {
-      const bool on = i0 + g < n_split && i0 + g != own;
+      const bool on = i0 + g < n_split;
       const float* si = row0 + static_cast<size_t>(i0 + g) * slot_elems;
       mv[g] = on ? __ldcg(si + static_cast<size_t>(d) * kRows) : -INFINITY;
       lv[g] = on ? __ldcg(si + static_cast<size_t>(d + 1) * kRows) : 0.f;
@@ -227,7 +227,7 @@ __device__ __forceinline__ void merge_stats(const float* row0, size_t slot_elems
     float mn = mr;
 #pragma unroll
     for (int g = 0; g < kMergeGroup; ++g) mn = fmaxf(mn, mv[g]);
-    ls *= ex2(mr - mn);  // every part's m is finite
+    ls *= ex2(mr - mn);  // 0 on the first group (mr = -inf); every part's m is finite
 #pragma unroll
     for (int g = 0; g < kMergeGroup; ++g) ls += ex2(mv[g] - mn) * lv[g];  // absent parts add 0
     mr = mn;
@@ -237,30 +237,23 @@ __device__ __forceinline__ void merge_stats(const float* row0, size_t slot_elems
 }
 
 // Columns c_begin .. c_begin + NCOLS - 1 of the merged row to bf16 at dst (which points at
-// column c_begin of the output row), 16 at a time; tO is the TMEM address of the merger's own
-// O at column c_begin (this thread's lane), w_own its weight 2^(m_own - mref) / sum.  Warp-
-// collective (TMEM loads).  NCOLS is a multiple of 8; TMEM holds O padded to 16 columns.
-template <int NCOLS>
+// column c_begin of the output row), CB at a time.  NCOLS and CB are multiples of 8.
+template <int NCOLS, int CB = 16>
 __device__ __forceinline__ void merge_columns(const float* row0, size_t slot_elems, int d, int n_split,
-                                              int own, int c_begin, uint32_t tO, float w_own,
-                                              float mref, float inv, uint16_t* dst, bool in_range) {
-  static_assert(NCOLS % 8 == 0, "whole 16-byte stores");
-  constexpr int CB = 16;
+                                              int c_begin, float mref, float inv, uint16_t* dst,
+                                              bool in_range) {
+  static_assert(NCOLS % 8 == 0 && CB % 8 == 0, "whole 16-byte stores");
 #pragma unroll
   for (int cb = 0; cb < NCOLS; cb += CB) {
     const int nc = NCOLS - cb < CB ? NCOLS - cb : CB;  // constant once unrolled
-    uint32_t o[CB];
-    tmem_ld16(tO + static_cast<uint32_t>(cb), o);
-    tmem_wait_ld();
-    reg_fence<CB>(o);
     float acc[CB];
 #pragma unroll
-    for (int k = 0; k < CB; ++k) acc[k] = w_own * __uint_as_float(o[k]);
+    for (int k = 0; k < CB; ++k) acc[k] = 0.f;
     for (int i0 = 0; i0 < n_split; i0 += kMergeGroup) {
       float v[kMergeGroup][CB], mv[kMergeGroup];
 #pragma unroll
       for (int g = 0; g < kMergeGroup; ++g) {
-        const bool on = i0 + g < n_split && i0 + g != own;
+        const bool on = i0 + g < n_split;
         const float* si = row0 + static_cast<size_t>(i0 + g) * slot_elems;
         mv[g] = on ? __ldcg(si + static_cast<size_t>(d) * kRows) : -INFINITY;
 #pragma unroll
@@ -410,22 +403,16 @@ __device__ __forceinline__ CtaWork cta_work(const AttnParams& p) {
   return w;
 }
 
-// After a merge: mark the other parts' slots of the query tile dead in L2 (the merger's own
-// slot was never written), so they are dropped instead of written back to DRAM.
+// After a merge: mark every part's slot of the query tile dead in L2, so the partials are
+// dropped instead of written back to DRAM.
 template <int D>
-__device__ __forceinline__ void discard_partials(const float* slot0, int n_split, int own, int tid,
-                                                 int nthreads) {
+__device__ __forceinline__ void discard_partials(const float* slot0, int n_split, int tid, int nthreads) {
   static_assert((D + 2) * kRows * 4 % 128 == 0, "slots are whole 128-byte lines");
-  constexpr int kLines = (D + 2) * kRows * 4 / 128;  // per slot
   const char* base = reinterpret_cast<const char*>(slot0);
   // the workspace only has to be 16-byte aligned: skip when the lines are not whole
   if ((reinterpret_cast<uintptr_t>(base) & 127u) != 0) return;
-  const int lines = (n_split - 1) * kLines;
-  for (int i = tid; i < lines; i += nthreads) {
-    const int slot = i / kLines;
-    const int idx = (slot >= own ? slot + 1 : slot) * kLines + (i - slot * kLines);
-    discard_l2_line(base + static_cast<size_t>(idx) * 128);
-  }
+  const int lines = n_split * (D + 2) * kRows * 4 / 128;
+  for (int i = tid; i < lines; i += nthreads) discard_l2_line(base + static_cast<size_t>(i) * 128);
 }
 
 // ------------------------------------------------------------------ head_dim 64: half rows
@@ -594,8 +581,11 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
   Segments seg;
   seg.init(p);
   const int n_all = seg.total();
-  const int j0 = static_cast<int>(static_cast<long long>(part) * n_all / p.n_split);
-  const int j1 = static_cast<int>(static_cast<long long>(part + 1) * n_all / p.n_split);
+  // part r takes context tiles [ceil(r n / k), ceil((r + 1) n / k)): the first parts take the
+  // extra tiles, and part 0 starts with the fresh rows, which it may compute before the
+  // previous micro-step has finished with the buffer
+  const int j0 = static_cast<int>((static_cast<long long>(part) * n_all + p.n_split - 1) / p.n_split);
+  const int j1 = static_cast<int>((static_cast<long long>(part + 1) * n_all + p.n_split - 1) / p.n_split);
   const int n_tiles = j1 - j0;  // this CTA's context tiles: j0 .. j1-1
 
   if (warp >= 16) {
@@ -890,15 +880,17 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
           unsigned* cnt = p.ws_cnt + (static_cast<size_t>(pair) * 2 + t) * 2;  // arrived, written
           if (hh == 0 && rloc == 0) s_last[t] = atomicAdd(cnt, 1u) == static_cast<unsigned>(p.n_split - 1);
           named_bar_sync(9 + t, 2 * kRows);
-          if (!s_last[t]) {
-            // partial: O row (64 columns, this thread's 32), m, l into this part's slot, column-major
-            float* mine = slot0 + static_cast<size_t>(part) * slot_elems;
+          // every part stores its partial (O row: this thread's 32 of the 64 columns; m, l),
+          // column-major -- the merger too, so that the merge reads all parts in part order
+          // whichever part merges
+          float* mine = slot0 + static_cast<size_t>(part) * slot_elems;
 #pragma unroll
-            for (int k = 0; k < 32; ++k) mine[(32 * hh + k) * kRows + rloc] = o[k];
-            if (hh == 0) {
-              mine[D * kRows + rloc] = m;
-              mine[(D + 1) * kRows + rloc] = lrow;
-            }
+          for (int k = 0; k < 32; ++k) mine[(32 * hh + k) * kRows + rloc] = o[k];
+          if (hh == 0) {
+            mine[D * kRows + rloc] = m;
+            mine[(D + 1) * kRows + rloc] = lrow;
+          }
+          if (!s_last[t]) {
             __threadfence();
             named_bar_sync(9 + t, 2 * kRows);
             PF_TRACE_EV(3);
@@ -906,7 +898,7 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
           } else {
             // the merger: wait (bounded) for the other parts' partials -- they have all arrived,
             // so they are running and wait for nothing -- then reset the counters for the next
-            // launch and combine them with its own part, which it never stores
+            // launch; its own partial is visible to its threads after the barrier
             if (hh == 0 && rloc == 0) {
               const bool ready = wait_count_geq(cnt + 1, static_cast<unsigned>(p.n_split - 1), abort, kWaitNs);
               if (ready) {
@@ -922,14 +914,13 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
             if (s_last[2 + t]) {
               // this thread's 32 columns of its row
               float mref, inv;
-              merge_stats(slot0 + rloc, slot_elems, D, p.n_split, part, m, lrow, mref, inv);
-              merge_columns<32>(slot0 + rloc, slot_elems, D, p.n_split, part, 32 * hh, tO,
-                                ex2(m - mref) * inv, mref, inv, dst, in_range);
+              merge_stats(slot0 + rloc, slot_elems, D, p.n_split, mref, inv);
+              merge_columns<32, 8>(slot0 + rloc, slot_elems, D, p.n_split, 32 * hh, mref, inv, dst, in_range);
               PF_TRACE_EV(5);
               if (p.discard) {
-                // every thread of the tile has read the other parts' slots: drop them from L2
+                // every thread of the tile has read all parts' slots: drop them from L2
                 named_bar_sync(9 + t, 2 * kRows);
-                discard_partials<D>(slot0, p.n_split, part, hh * kRows + rloc, 2 * kRows);
+                discard_partials<D>(slot0, p.n_split, hh * kRows + rloc, 2 * kRows);
               }
             }
           }
@@ -1035,28 +1026,30 @@ __device__ __forceinline__ void full_row_epilogue(const AttnParams& p, uint32_t 
   unsigned* cnt = p.ws_cnt + (static_cast<size_t>(pair) * 2 + t) * 2;  // arrived, written
   if (rloc == 0) s_last[t] = atomicAdd(cnt, 1u) == static_cast<unsigned>(p.n_split - 1);
   named_bar_sync(1 + t, kRows);
+  // every part stores its partial, O row (d columns), m, l, column-major -- the merger too,
+  // so that the merge reads all parts in part order whichever part merges
+  float* mine = slot0 + static_cast<size_t>(part) * slot_elems;
+#pragma unroll
+  for (int c0 = 0; c0 < kMmaN; c0 += 16) {
+    uint32_t o[16];
+    tmem_ld16(tO + c0, o);
+    tmem_wait_ld();
+    reg_fence<16>(o);
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      if (c0 + k < D) mine[(c0 + k) * kRows + rloc] = __uint_as_float(o[k]);
+  }
+  mine[D * kRows + rloc] = m;
+  mine[(D + 1) * kRows + rloc] = l;
   if (!s_last[t]) {
-    // partial: O row (d columns), m, l into this part's slot, column-major
-    float* mine = slot0 + static_cast<size_t>(part) * slot_elems;
-#pragma unroll
-    for (int c0 = 0; c0 < kMmaN; c0 += 16) {
-      uint32_t o[16];
-      tmem_ld16(tO + c0, o);
-      tmem_wait_ld();
-      reg_fence<16>(o);
-#pragma unroll
-      for (int k = 0; k < 16; ++k)
-        if (c0 + k < D) mine[(c0 + k) * kRows + rloc] = __uint_as_float(o[k]);
-    }
-    mine[D * kRows + rloc] = m;
-    mine[(D + 1) * kRows + rloc] = l;
     __threadfence();
     named_bar_sync(1 + t, kRows);
     if (rloc == 0) atomicAdd(cnt + 1, 1u);
     return;
   }
   // the merger: wait until the other parts' partials are written, then reset the counters
-  // for the next launch (every other part has counted both by then)
+  // for the next launch (every other part has counted both by then); its own partial is
+  // visible to its threads after the barrier
   if (rloc == 0) {
     const bool ready = wait_count_geq(cnt + 1, static_cast<unsigned>(p.n_split - 1), abort, kWaitNs);
     if (ready) {
@@ -1070,13 +1063,12 @@ __device__ __forceinline__ void full_row_epilogue(const AttnParams& p, uint32_t 
   named_bar_sync(1 + t, kRows);
   if (!s_last[2 + t]) return;
   float mref, inv;
-  merge_stats(slot0 + rloc, slot_elems, D, p.n_split, part, m, l, mref, inv);
-  merge_columns<D>(slot0 + rloc, slot_elems, D, p.n_split, part, 0, tO, ex2(m - mref) * inv, mref, inv,
-                   dst, in_range);
+  merge_stats(slot0 + rloc, slot_elems, D, p.n_split, mref, inv);
+  merge_columns<D>(slot0 + rloc, slot_elems, D, p.n_split, 0, mref, inv, dst, in_range);
   if (p.discard) {
-    // every thread of the tile has read the other parts' slots: drop them from L2
+    // every thread of the tile has read all parts' slots: drop them from L2
     named_bar_sync(1 + t, kRows);
-    discard_partials<D>(slot0, p.n_split, part, rloc, kRows);
+    discard_partials<D>(slot0, p.n_split, rloc, kRows);
   }
 }
 
@@ -1182,8 +1174,11 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
   Segments seg;
   seg.init(p);
   const int n_all = seg.total();
-  const int j0 = static_cast<int>(static_cast<long long>(part) * n_all / p.n_split);
-  const int j1 = static_cast<int>(static_cast<long long>(part + 1) * n_all / p.n_split);
+  // part r takes context tiles [ceil(r n / k), ceil((r + 1) n / k)): the first parts take the
+  // extra tiles, and part 0 starts with the fresh rows, which it may compute before the
+  // previous micro-step has finished with the buffer
+  const int j0 = static_cast<int>((static_cast<long long>(part) * n_all + p.n_split - 1) / p.n_split);
+  const int j1 = static_cast<int>((static_cast<long long>(part + 1) * n_all + p.n_split - 1) / p.n_split);
   const int n_tiles = j1 - j0;  // this CTA's context tiles: j0 .. j1-1
 
   if (warp >= 8) {
