@@ -145,16 +145,22 @@ pf_status pf_text_attn_step(pf_ctx* ctx, int layer, const void* q_txt, const voi
 pf_status pf_qk_rmsnorm(void* x, int64_t n_vectors, int head_dim, const void* gain, float eps,
                         void* stream);
 
-/* Bytes of the optional attention workspace for this configuration (0 if cfg is invalid).
- * With a workspace set, a call may split each query tile's key range over several CTAs so
- * that the grid fills the GPU's SMs in near-whole waves; the parts are merged exactly in
- * the log-sum-exp sense (rescaled by their row maxima) by the last part to finish. */
+/* Bytes of the optional attention workspace for this configuration (0 if cfg is invalid, or
+ * if no call of the configuration would split).  With a workspace set, a call may split each
+ * query tile's key range over several CTAs so that the grid fills the GPU's SMs in near-whole
+ * waves; the parts are merged exactly in the log-sum-exp sense (rescaled by their row maxima)
+ * by the last part to finish.  The workspace also holds per-layer ordering counters: a call
+ * reads a layer's buffer once the earlier calls on that layer have scattered into it, and
+ * scatters once they have finished reading it, so consecutive calls on different layers of
+ * one stream overlap on the GPU (without a workspace, each call waits for the previous one
+ * before it touches the buffer). */
 size_t pf_workspace_bytes(const pf_config* cfg);
 
 /* Attach a caller-owned device workspace (16-byte aligned, >= pf_workspace_bytes(cfg))
  * to ctx and zero its counters on `stream`.  ws = NULL detaches it (no key-range split).
- * Calls that share a workspace must not run concurrently (one workspace per stream).
- * After PF_ERR_TIMEOUT, set the workspace again to re-zero the counters. */
+ * Calls that share a workspace must not run concurrently (one workspace per stream), and the
+ * calls of a context run on that one stream.  After PF_ERR_TIMEOUT, set the workspace again
+ * to re-zero the counters. */
 pf_status pf_set_workspace(pf_ctx* ctx, void* ws, size_t ws_bytes, void* stream);
 
 /* Next patch index the layer expects (0 at the start of a step).  Checkpoint helper: a

@@ -125,7 +125,8 @@ constexpr uint32_t kColO = 256;        // split-tile kernel: O_t at column 256 +
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kMaxSplit = 16;          // most key-range parts per query tile
 
-enum : unsigned { kWdLoad = 1u, kWdMma = 2u, kWdSoftmax = 4u, kWdEpilogue = 8u, kWdSelftest = 16u };
+enum : unsigned { kWdLoad = 1u, kWdMma = 2u, kWdSoftmax = 4u, kWdEpilogue = 8u, kWdSelftest = 16u,
+                  kWdScatter = 32u };
 
 template <int D>
 struct Dims {
@@ -341,8 +342,16 @@ __device__ __forceinline__ void raise_abort(volatile int* abort, unsigned code) 
 template <int D>
 __device__ __forceinline__ void scatter_share(const AttnParams& p, int lane) {
   if (p.k_dst == nullptr) return;
-  // the previous micro-step reads these buffer rows (as stale context): wait for it
-  grid_dep_wait();
+  // earlier calls on the layer read these buffer rows (as stale context): wait until every
+  // CTA of theirs has finished reading (or, without counters, for the previous grid)
+  if (p.dep_read != nullptr) {
+    if (!wait_count_geq64(p.dep_read, p.dep_read_target, nullptr, kWaitNs)) {
+      if (lane == 0) atomicOr(&g_watchdog, kWdScatter);
+      return;
+    }
+  } else {
+    grid_dep_wait();
+  }
   const long long per_b = static_cast<long long>(p.plen) * p.heads * D / 8;  // 16-byte vectors
   const long long total = per_b * p.batch;
   const long long lo = total * blockIdx.x / gridDim.x;
@@ -374,6 +383,12 @@ __device__ __forceinline__ void scatter_share(const AttnParams& p, int lane) {
         vdst[i1 + shift] = v1;
       }
     }
+  }
+  if (p.dep_scat != nullptr) {
+    // this CTA's share is in the buffer: count it for later calls on the layer
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) count_release(p.dep_scat);
   }
 }
 
@@ -604,8 +619,16 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
           int src, row0, nv;
           seg.tile(j0 + j, src, row0, nv);
           if ((src == 1 || src == 3) && !dep_done) {
-            // buffer rows: the previous micro-step's scatter writes some of them
-            grid_dep_wait();
+            // buffer rows: wait until every earlier call on the layer has scattered into the
+            // buffer (or, without counters, for the previous grid)
+            if (p.dep_scat != nullptr) {
+              if (!wait_count_geq64(p.dep_scat, p.dep_scat_target, abort, kWaitNs)) {
+                ok = false;
+                break;
+              }
+            } else {
+              grid_dep_wait();
+            }
             dep_done = true;
           }
           for (int kv = 0; kv < 2; ++kv) {
@@ -630,6 +653,8 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
         mbar_wait(qbar, 0, nullptr, kWaitNs);
         for (int i = issued > S ? issued - S : 0; i < issued; ++i)
           mbar_wait(smem_u32(kv_full + (i % S)), (i / S) & 1, nullptr, kWaitNs);
+        // this CTA has read all it reads of the buffer: count it for later calls' scatters
+        if (p.dep_read != nullptr) count_release(p.dep_read);
       }
     } else if (warp == kHrWarpMma0 || (NQ == 2 && warp == kHrWarpMma1)) {
       // ------------------------------------------------------------ MMA issuer of query tile t
@@ -1199,8 +1224,16 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
           int src, row0, nv;
           seg.tile(j0 + j, src, row0, nv);
           if ((src == 1 || src == 3) && !dep_done) {
-            // buffer rows: the previous micro-step's scatter writes some of them
-            grid_dep_wait();
+            // buffer rows: wait until every earlier call on the layer has scattered into the
+            // buffer (or, without counters, for the previous grid)
+            if (p.dep_scat != nullptr) {
+              if (!wait_count_geq64(p.dep_scat, p.dep_scat_target, abort, kWaitNs)) {
+                ok = false;
+                break;
+              }
+            } else {
+              grid_dep_wait();
+            }
             dep_done = true;
           }
           for (int kv = 0; kv < 2; ++kv) {
@@ -1227,6 +1260,8 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
         mbar_wait(qbar, 0, nullptr, kWaitNs);
         for (int i = issued > S ? issued - S : 0; i < issued; ++i)
           mbar_wait(smem_u32(kv_full + (i % S)), (i / S) & 1, nullptr, kWaitNs);
+        // this CTA has read all it reads of the buffer: count it for later calls' scatters
+        if (p.dep_read != nullptr) count_release(p.dep_read);
       }
     } else if (warp == kWarpMma || (NQ == 2 && warp == kWarpMma2)) {
       // ------------------------------------------------------------ MMA issuer of query tile t

@@ -30,6 +30,10 @@ struct pf_ctx {
   uint8_t* ws = nullptr;         // optional attention workspace (caller-owned)
   size_t ws_bytes = 0;
   int n_sms = 0;                 // queried on first use
+  // per layer: the CTAs of the calls launched so far that will count a finished scatter /
+  // finished buffer reads on the workspace's ordering counters (reset with the workspace)
+  std::vector<unsigned long long> scat_target;
+  std::vector<unsigned long long> read_target;
 };
 
 namespace {
@@ -122,12 +126,18 @@ constexpr int kAssumedSms = 148;
 
 // Counters first (fixed place, sized for the larger of patch and text-query calls), then the
 // partial slots.
-// Two counters (parts arrived, partials written) per query tile of every pair.
-size_t counter_bytes(int pairs) { return ((static_cast<size_t>(pairs) * 2 * 2 * 4 + 255) / 256) * 256; }
+// Two counters (parts arrived, partials written) per query tile of every pair, then two 64-bit
+// ordering counters (CTAs that finished their scatter, CTAs that finished reading the buffer)
+// per layer.
+size_t pair_counter_bytes(int pairs) { return static_cast<size_t>(pairs) * 2 * 2 * 4; }
+size_t counter_bytes(const pf_config& c) {
+  const size_t b = pair_counter_bytes(pairs_of(c)) + static_cast<size_t>(c.n_layers) * 2 * 8;
+  return ((b + 255) / 256) * 256;
+}
 
 size_t workspace_for(const pf_config& c, int n_sms) {
   const int plen = c.n_img / c.n_patches;
-  const size_t cb = counter_bytes(pairs_of(c));
+  const size_t cb = counter_bytes(c);
   size_t best = 0;
   auto consider = [&](int q_rows, int tiles) {
     const int pairs = pairs_for(c, q_rows);
@@ -147,7 +157,7 @@ bool layer_ok(const pf_ctx* ctx, int layer) { return layer >= 0 && layer < ctx->
 
 // Fill the fields common to every attention call (sizes, scale, work decomposition and
 // key-range split) and launch.  p carries the tensor maps, pointers and segments.
-cudaError_t launch_attention(pf_ctx* ctx, pf::AttnParams& p, void* stream) {
+cudaError_t launch_attention(pf_ctx* ctx, pf::AttnParams& p, int layer, void* stream) {
   const pf_config& c = ctx->cfg;
   p.batch = c.batch;
   p.heads = c.heads;
@@ -169,7 +179,7 @@ cudaError_t launch_attention(pf_ctx* ctx, pf::AttnParams& p, void* stream) {
         ctx->n_sms = kAssumedSms;
     }
     const int tiles = pf::attn_context_tiles(p.fresh_rows, p.lo_len, p.hi_len, c.n_txt);
-    const size_t cb = counter_bytes(pairs_of(c));
+    const size_t cb = counter_bytes(c);
     int cap = 1;  // most parts the workspace can hold
     while (cap < 16 && cb + pf::attn_workspace_bytes(p.n_pairs, c.head_dim, cap + 1) <= ctx->ws_bytes)
       ++cap;
@@ -183,7 +193,24 @@ cudaError_t launch_attention(pf_ctx* ctx, pf::AttnParams& p, void* stream) {
       p.discard = static_cast<long long>(p.n_pairs) * p.n_split > ctx->n_sms ? 1 : 0;
     }
   }
-  return pf::launch_patch_attn(p, static_cast<cudaStream_t>(stream));
+  if (ctx->ws != nullptr) {
+    // order against the other calls on this layer through the workspace's counters, so that
+    // the launch need not wait for the previous grid (often another layer's) before it reads
+    unsigned long long* dep = reinterpret_cast<unsigned long long*>(
+        ctx->ws + pair_counter_bytes(pairs_of(c))) + static_cast<size_t>(layer) * 2;
+    p.dep_scat = dep;
+    p.dep_read = dep + 1;
+    p.dep_scat_target = ctx->scat_target[layer];
+    p.dep_read_target = ctx->read_target[layer];
+  }
+  const cudaError_t e = pf::launch_patch_attn(p, static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess && ctx->ws != nullptr) {
+    // every CTA of this launch counts itself once on each counter it takes part in
+    const unsigned long long ctas = static_cast<unsigned long long>(p.n_pairs) * p.n_split;
+    ctx->read_target[layer] += ctas;
+    if (p.k_dst != nullptr) ctx->scat_target[layer] += ctas;
+  }
+  return e;
 }
 
 // K/V regions of a layer's buffer: half 0 is [K | V]; DistriFusion adds half 1 [K | V].
@@ -326,7 +353,7 @@ pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
   p.lo_len = lo_len;
   p.hi_row0 = (patch + 1) * plen;
   p.hi_len = c.n_img - (patch + 1) * plen;
-  const pf_status ls = from_attn_launch(launch_attention(ctx, p, stream));
+  const pf_status ls = from_attn_launch(launch_attention(ctx, p, layer, stream));
   if (ls != PF_OK) return ls;
 
   if (pipefusion) {
@@ -372,7 +399,7 @@ pf_status pf_text_attn_step(pf_ctx* ctx, int layer, const void* q_txt, const voi
   p.lo_len = c.n_img;   // the whole buffer as it stands
   p.hi_row0 = c.n_img;
   p.hi_len = 0;
-  const pf_status ls = from_attn_launch(launch_attention(ctx, p, stream));
+  const pf_status ls = from_attn_launch(launch_attention(ctx, p, layer, stream));
   if (ls != PF_OK) return ls;
   return PF_OK;
 }
@@ -416,12 +443,14 @@ pf_status pf_set_workspace(pf_ctx* ctx, void* ws, size_t ws_bytes, void* stream)
     return PF_OK;
   }
   if (!aligned16(ws)) return PF_ERR_ALIGN;
-  const size_t cb = counter_bytes(pairs_of(ctx->cfg));
+  const size_t cb = counter_bytes(ctx->cfg);
   if (ws_bytes < cb) return PF_ERR_INVALID_ARG;
   cudaError_t e = pf::launch_zero_u32(static_cast<unsigned*>(ws), cb / 4, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return PF_ERR_CUDA;
   ctx->ws = static_cast<uint8_t*>(ws);
   ctx->ws_bytes = ws_bytes;
+  ctx->scat_target.assign(ctx->cfg.n_layers, 0ull);
+  ctx->read_target.assign(ctx->cfg.n_layers, 0ull);
   return PF_OK;
 }
 

@@ -43,6 +43,16 @@ struct AttnParams {
   float* ws_part;       // partial (O, m, l) slots, [pair][tile][part][d + 2][128] fp32
   unsigned* ws_cnt;     // per [pair][tile]: parts arrived, partials written; zero between launches
   int discard;          // drop the merged partials from L2 (1) rather than let them be written back
+  // Order against the other calls on the same layer buffer without waiting for the whole
+  // previous grid: the buffer is read once *dep_scat (CTAs of earlier calls on the layer that
+  // finished their scatter) reaches dep_scat_target, and the scatter writes once *dep_read
+  // (CTAs of earlier calls on the layer that finished reading the buffer) reaches
+  // dep_read_target.  Every CTA counts itself on both when done.  Null: wait for the previous
+  // grid instead (griddepcontrol.wait).
+  unsigned long long* dep_scat;
+  unsigned long long* dep_read;
+  unsigned long long dep_scat_target;
+  unsigned long long dep_read_target;
 };
 
 // Query tiles per CTA chosen for a patch length (1 or 2).

@@ -117,6 +117,31 @@ __device__ __forceinline__ bool wait_count_geq(const unsigned* c, unsigned targe
   }
 }
 
+// The same for a 64-bit counter, with a proxy fence after it so that TMA loads (the async
+// proxy) issued afterwards see what the counted writers stored.
+__device__ __forceinline__ bool wait_count_geq64(const unsigned long long* c, unsigned long long target,
+                                                 const volatile int* abort, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(c) : "memory");
+    if (v >= target) {
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      return true;
+    }
+    if (abort != nullptr && *abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+    __nanosleep(200);
+  }
+}
+
+// Count one event on a 64-bit counter with release semantics (what this thread -- and, through
+// a preceding fence or barrier, its peers -- wrote or finished reading is ordered before it).
+__device__ __forceinline__ void count_release(unsigned long long* c) {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(c) : "memory");
+}
+
 // ------------------------------------------------------------------ programmatic dependent launch
 
 // Let the next grid on the stream (launched with programmatic stream serialization) start

@@ -5,8 +5,9 @@ previous micro-step finishes and wait before they touch the K/V buffer, the outp
 workspace).  The other parity tests synchronise after every call to check the buffer; here
 every call of a few diffusion steps is enqueued first, each into its own output, and only then
 checked: sampled rows of every call against the fp64 oracle, the buffer against the last step,
-the device status word (a bounded wait that gave up would show as PF_ERR_TIMEOUT) and the
-key-range split's counters, which must all be back at zero.
+the device status word (a bounded wait that gave up would show as PF_ERR_TIMEOUT), the
+key-range split's counters, which must all be back at zero, and the per-layer ordering
+counters, which must agree.
 """
 import numpy as np
 import pytest
@@ -44,10 +45,16 @@ def test_overlapped_micro_steps_match_the_oracle(d):
                     outs[(s, l, p)] = pat.step(l, p, q, k, v, t["k_txt"], t["v_txt"])
         torch.cuda.synchronize()
         pat.check()  # no bounded wait gave up
-        # between launches every split counter (parts arrived, partials written) is back at 0:
-        # the merger of each query tile resets them once all parts have counted
+        # between launches every split counter (parts arrived, partials written: two per query
+        # tile of each of the B * H * 2 query-tile pairs) is back at 0, the merger of each query
+        # tile resets them; the per-layer ordering counters that follow count, for every CTA of
+        # every call, one finished scatter and one finished read of the buffer: equal after
+        # patch calls only, and non-zero
         assert pat.workspace is not None
-        assert int(pat.workspace[:256].count_nonzero()) == 0
+        pairs = wl.batch * wl.heads * 2
+        assert int(pat.workspace[:pairs * 16].count_nonzero()) == 0
+        order = pat.workspace[pairs * 16:pairs * 16 + L * 16].view(torch.int64).view(L, 2)
+        assert torch.equal(order[:, 0], order[:, 1]) and bool((order > 0).all()), order
         rng = np.random.default_rng(3)
         for (s, l, p), o in outs.items():
             cur, prev = steps[s][l], steps[max(s - 1, 0)][l]
