@@ -782,7 +782,7 @@ def main():
     ap.add_argument("--profile-norm", action="store_true",
                     help="only run two RMS normalisations of a full-spatial Q of the workload (for ncu)")
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=12)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="patchattn", choices=["patchattn", "reference"])
     ap.add_argument("--workload", default="flux", choices=sorted(synth.ATTN_WORKLOADS))
