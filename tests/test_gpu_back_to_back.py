@@ -1,13 +1,15 @@
 """Micro-steps launched back to back, with no host synchronisation between them.
 
-Consecutive attention launches overlap on the GPU (a launch's CTAs may start while the
-previous micro-step finishes and wait before they touch the K/V buffer, the output or the
-workspace).  The other parity tests synchronise after every call to check the buffer; here
-every call of a few diffusion steps is enqueued first, each into its own output, and only then
-checked: sampled rows of every call against the fp64 oracle, the buffer against the last step,
-the device status word (a bounded wait that gave up would show as PF_ERR_TIMEOUT), the
-key-range split's counters, which must all be back at zero, and the per-layer ordering
-counters, which must agree.
+Consecutive attention launches overlap on the GPU: a launch's CTAs may start while earlier
+micro-steps finish, and calls on the same layer buffer are ordered only by per-layer counters
+in the workspace (a call reads the buffer once the earlier calls on the layer have scattered
+into it, and scatters once they have finished reading it).  The other parity tests synchronise
+after every call to check the buffer; here every call of a few diffusion steps -- the patch
+calls of every layer, then text-token queries on every layer at the end of each step -- is
+enqueued first, each into its own output, and only then checked: sampled rows of every call
+against the fp64 oracle, the buffer against the last step, the device status word (a bounded
+wait that gave up would show as PF_ERR_TIMEOUT), the key-range split's counters, which must
+all be back at zero, and the per-layer ordering counters.
 """
 import numpy as np
 import pytest
@@ -20,16 +22,20 @@ from tests._oracle_util import f64
 
 pytestmark = pytest.mark.gpu
 
+PF, DF = pa.PF_SCHED_PIPEFUSION, pa.PF_SCHED_DISTRIFUSION
 
-@pytest.mark.parametrize("d", [64, 72, 128])
-def test_overlapped_micro_steps_match_the_oracle(d):
+
+@pytest.mark.parametrize("d,schedule", [(64, PF), (72, PF), (128, PF), (64, DF), (128, DF)])
+def test_overlapped_micro_steps_match_the_oracle(d, schedule):
     wl = synth.AttnWorkload("b2b", batch=1, heads=4, head_dim=d, grid_h=64, grid_w=64,
                             n_patches=8, n_txt=77, n_layers=2, n_steps=3, ar_a=0.95, ar_b=0.3)
-    S, L, M, P = wl.n_steps, wl.n_layers, wl.n_patches, wl.patch_len
+    S, L, M, P, T = wl.n_steps, wl.n_layers, wl.n_patches, wl.patch_len, wl.n_txt
     gen = synth.AttnInputs(wl, seed=21, device="cuda")
     steps = [[gen.step_tensors(l) for l in range(L)] for _ in range(S)]
-    pat = pa.PatchAttention(1, wl.heads, d, wl.n_img, M, wl.n_txt, L)
-    outs = {}
+    g = torch.Generator(device="cuda").manual_seed(5)
+    q_txt = [torch.randn(1, T, wl.heads, d, device="cuda", generator=g).bfloat16() for _ in range(L)]
+    pat = pa.PatchAttention(1, wl.heads, d, wl.n_img, M, T, L, schedule=schedule)
+    outs, txt_outs = {}, {}
     try:
         for l in range(L):
             pat.init_layer(l, steps[0][l]["k"], steps[0][l]["v"])
@@ -43,33 +49,49 @@ def test_overlapped_micro_steps_match_the_oracle(d):
                     q, k, v = patches[s][l][p]
                     t = steps[s][l]
                     outs[(s, l, p)] = pat.step(l, p, q, k, v, t["k_txt"], t["v_txt"])
+            for l in range(L):
+                t = steps[s][l]
+                txt_outs[(s, l)] = pat.text_step(l, q_txt[l], t["k_txt"], t["v_txt"])
         torch.cuda.synchronize()
         pat.check()  # no bounded wait gave up
-        # between launches every split counter (parts arrived, partials written: two per query
-        # tile of each of the B * H * 2 query-tile pairs) is back at 0, the merger of each query
-        # tile resets them; the per-layer ordering counters that follow count, for every CTA of
-        # every call, one finished scatter and one finished read of the buffer: equal after
-        # patch calls only, and non-zero
-        assert pat.workspace is not None
-        pairs = wl.batch * wl.heads * 2
-        assert int(pat.workspace[:pairs * 16].count_nonzero()) == 0
-        order = pat.workspace[pairs * 16:pairs * 16 + L * 16].view(torch.int64).view(L, 2)
-        assert torch.equal(order[:, 0], order[:, 1]) and bool((order > 0).all()), order
         rng = np.random.default_rng(3)
+        attention = oracle.patch_attention if schedule == PF else oracle.distrifusion_attention
         for (s, l, p), o in outs.items():
             cur, prev = steps[s][l], steps[max(s - 1, 0)][l]
             rows = sorted(set([0, P - 1] + list(rng.integers(0, P, 6))))
             h = int(rng.integers(0, wl.heads))
             take = lambda x: f64(x[0][:, h:h + 1])
-            ref = oracle.patch_attention(take(cur["q"]), take(cur["k"]), take(cur["v"]), take(prev["k"]),
-                                         take(prev["v"]), take(cur["k_txt"]), take(cur["v_txt"]), p, M,
-                                         wl.softmax_scale, rows=rows)
+            ref = attention(take(cur["q"]), take(cur["k"]), take(cur["v"]), take(prev["k"]),
+                            take(prev["v"]), take(cur["k_txt"]), take(cur["v_txt"]), p, M,
+                            wl.softmax_scale, rows=rows)
             got = f64(o[0][rows][:, h:h + 1])
             rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
             assert rel <= 5e-3, (s, l, p, rel)
+        for (s, l), o in txt_outs.items():
+            # after a step's last patch the buffer holds that step's K/V under both schedules
+            cur = steps[s][l]
+            h = int(rng.integers(0, wl.heads))
+            rows = sorted(set([0, T - 1] + list(rng.integers(0, T, 6))))
+            take = lambda x: f64(x[0][:, h:h + 1])
+            ref = oracle.attend(take(q_txt[l])[rows], np.concatenate([take(cur["k"]), take(cur["k_txt"])]),
+                                np.concatenate([take(cur["v"]), take(cur["v_txt"])]), wl.softmax_scale)
+            got = f64(o[0][rows][:, h:h + 1])
+            rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+            assert rel <= 5e-3, (s, l, "text", rel)
         for l in range(L):
-            kb, vb = pat.buffer_kv(l)
-            assert torch.equal(kb.view(torch.int16), steps[-1][l]["k"].view(torch.int16))
-            assert torch.equal(vb.view(torch.int16), steps[-1][l]["v"].view(torch.int16))
+            last_k, last_v = steps[-1][l]["k"].view(torch.int16), steps[-1][l]["v"].view(torch.int16)
+            halves = (0,) if schedule == PF else (0, 1)
+            assert any(torch.equal(pat.buffer_kv(l, hf)[0].view(torch.int16), last_k) and
+                       torch.equal(pat.buffer_kv(l, hf)[1].view(torch.int16), last_v) for hf in halves), l
+        # between launches every split counter (parts arrived, partials written: two per query
+        # tile of each of the B * H * 2 patch query-tile pairs, which outnumber the text
+        # queries' pairs) is back at 0, the merger of each query tile resets them; the per-layer
+        # ordering counters that follow count, for every CTA of every call, one finished read of
+        # the buffer, and for every CTA of a patch call one finished scatter
+        assert pat.workspace is not None
+        pairs = wl.batch * wl.heads * 2
+        assert int(pat.workspace[:pairs * 16].count_nonzero()) == 0
+        order = pat.workspace[pairs * 16:pairs * 16 + L * 16].view(torch.int64).view(L, 2)
+        assert bool((order[:, 0] > 0).all()) and bool((order[:, 1] > order[:, 0]).all()), order
     finally:
         pat.close()
