@@ -1506,22 +1506,28 @@ int attn_context_tiles(int fresh_rows, int lo_len, int hi_len, int n_txt) {
 }
 
 int attn_choose_split(int n_pairs, int n_tiles, int n_sms, int max_split) {
-  // cost model in units of context tiles: whole waves of CTAs times the tiles per CTA plus
-  // a fixed per-CTA overhead (launch, TMEM allocation, Q load, pipeline fill, merge)
-  constexpr long long kOverheadTiles = 6;
-  int best = 1;
-  long long best_cost = -1;
+  // Cost model in units of context tiles.  Launches overlap on the GPU (the per-layer ordering
+  // counters let a launch start while earlier ones finish), so a call costs the larger of its
+  // share of SM time, n_pairs (n_tiles + k c) / n_sms, and half the length of one CTA,
+  // (ceil(n_tiles / k) + c) / 2: at most two launches on one layer buffer make progress at
+  // once (the next one reads after this one's scatter, scatters after this one's reads).  c is
+  // the fixed cost of a CTA (launch, TMEM allocation, Q load, pipeline fill, merge).  Of the
+  // splits within 5% of the cheapest the smallest is taken: fewer partials to store and merge.
+  constexpr double kOverheadTiles = 6.0;
   const int kmax = max_split < kMaxSplit ? max_split : kMaxSplit;
+  double cost[kMaxSplit + 1];
+  double best = -1.0;
+  int kn = 0;
   for (int k = 1; k <= kmax && k <= n_tiles; ++k) {
-    const long long ctas = static_cast<long long>(n_pairs) * k;
-    const long long waves = (ctas + n_sms - 1) / n_sms;
-    const long long cost = waves * ((n_tiles + k - 1) / k + kOverheadTiles);
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best = k;
-    }
+    const double sm_time = static_cast<double>(n_pairs) * (n_tiles + k * kOverheadTiles) / n_sms;
+    const double cta = 0.5 * ((n_tiles + k - 1) / k + kOverheadTiles);
+    cost[k] = sm_time > cta ? sm_time : cta;
+    if (best < 0.0 || cost[k] < best) best = cost[k];
+    kn = k;
   }
-  return best;
+  for (int k = 1; k <= kn; ++k)
+    if (cost[k] <= 1.05 * best) return k;
+  return 1;
 }
 
 size_t attn_workspace_bytes(int n_pairs, int head_dim, int n_split) {

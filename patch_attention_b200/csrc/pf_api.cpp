@@ -138,7 +138,7 @@ size_t counter_bytes(const pf_config& c) {
 size_t workspace_for(const pf_config& c, int n_sms) {
   const int plen = c.n_img / c.n_patches;
   const size_t cb = counter_bytes(c);
-  size_t best = 0;
+  size_t best = cb;  // the counters, split or not
   auto consider = [&](int q_rows, int tiles) {
     const int pairs = pairs_for(c, q_rows);
     const int k = pf::attn_choose_split(pairs, tiles, n_sms, 1 << 30);
