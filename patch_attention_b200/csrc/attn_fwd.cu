@@ -29,12 +29,16 @@
 // reference maximum for numerator and denominator.
 //
 // Work decomposition: one CTA per (pair, part), where a pair is one (batch, head, group of
-// NQ query tiles) and its context tiles are split into n_split contiguous parts so that
-// the grid fills the SMs in near-whole waves.  A part that does not cover the whole
-// context writes its unnormalised O row with its reference maximum m and sum l to a
-// workspace slot; the last part of a query tile to finish (an atomic counter decides, no
-// CTA ever waits for another) merges all parts, O = sum_i 2^(m_i - M) O_i / sum_i 2^(m_i - M) l_i,
-// and writes the bf16 output.
+// NQ query tiles) and its context tiles may be split into n_split contiguous parts (the
+// host picks n_split for launches that overlap their neighbours).  Every part of a split
+// writes its unnormalised O row with its reference maximum m and sum l to a workspace slot;
+// the last part of a query tile to arrive (an atomic counter decides) waits, bounded, for
+// the others' slots -- they have all arrived, so they are running -- and merges all parts
+// in part order, O = sum_i 2^(m_i - M) O_i / sum_i 2^(m_i - M) l_i, into the bf16 output.
+//
+// Ordering between launches: with a workspace, calls on one layer buffer are ordered by two
+// per-layer counters (CTAs that finished their scatter, CTAs that finished reading the
+// buffer) instead of by the completion of the previous grid, so that launches overlap.
 //
 // Every wait is bounded (2 s); on expiry the kernel records the role in a device word,
 // raises a CTA-wide abort flag, drains its in-flight copies and MMAs, frees TMEM and

@@ -47,7 +47,8 @@ struct AttnParams {
   // previous grid: the buffer is read once *dep_scat (CTAs of earlier calls on the layer that
   // finished their scatter) reaches dep_scat_target, and the scatter writes once *dep_read
   // (CTAs of earlier calls on the layer that finished reading the buffer) reaches
-  // dep_read_target.  Every CTA counts itself on both when done.  Null: wait for the previous
+  // dep_read_target.  Every CTA counts its finished reads, and its finished scatter share
+  // when the call scatters.  Null: wait for the previous
   // grid instead (griddepcontrol.wait).
   unsigned long long* dep_scat;
   unsigned long long* dep_read;
