@@ -97,3 +97,50 @@ def test_overlapped_micro_steps_match_the_oracle(d, schedule):
         assert bool((order > 0).all()) and bool((order[:, 1] > order[:, 0]).all()), order
     finally:
         pat.close()
+
+
+def test_workspace_detached_and_attached_between_steps():
+    """Calls without a workspace wait for the previous grid; attaching a workspace again zeroes
+    the counters (ordered after the calls still running on the stream) and restarts the host's
+    targets.  Steps alternate between the two, still without host synchronisation."""
+    d = 128
+    wl = synth.AttnWorkload("b2bws", batch=1, heads=2, head_dim=d, grid_h=32, grid_w=64,
+                            n_patches=4, n_txt=33, n_layers=2, n_steps=4, ar_a=0.95, ar_b=0.3)
+    S, L, M, P = wl.n_steps, wl.n_layers, wl.n_patches, wl.patch_len
+    gen = synth.AttnInputs(wl, seed=8, device="cuda")
+    steps = [[gen.step_tensors(l) for l in range(L)] for _ in range(S)]
+    pat = pa.PatchAttention(1, wl.heads, d, wl.n_img, M, wl.n_txt, L)
+    ws = pat.workspace
+    assert ws is not None
+    outs = {}
+    try:
+        for l in range(L):
+            pat.init_layer(l, steps[0][l]["k"], steps[0][l]["v"])
+        for s in range(S):
+            pa.pf_set_workspace(pat.ctx, ws if s % 2 == 0 else None)
+            for p in range(M):
+                for l in range(L):
+                    t = steps[s][l]
+                    sl = slice(p * P, (p + 1) * P)
+                    outs[(s, l, p)] = pat.step(l, p, t["q"][:, sl].contiguous(), t["k"][:, sl].contiguous(),
+                                               t["v"][:, sl].contiguous(), t["k_txt"], t["v_txt"])
+        torch.cuda.synchronize()
+        pat.check()
+        rng = np.random.default_rng(4)
+        for (s, l, p), o in outs.items():
+            cur, prev = steps[s][l], steps[max(s - 1, 0)][l]
+            rows = sorted(set([0, P - 1] + list(rng.integers(0, P, 6))))
+            h = int(rng.integers(0, wl.heads))
+            take = lambda x: f64(x[0][:, h:h + 1])
+            ref = oracle.patch_attention(take(cur["q"]), take(cur["k"]), take(cur["v"]), take(prev["k"]),
+                                         take(prev["v"]), take(cur["k_txt"]), take(cur["v_txt"]), p, M,
+                                         wl.softmax_scale, rows=rows)
+            got = f64(o[0][rows][:, h:h + 1])
+            rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+            assert rel <= 5e-3, (s, l, p, rel)
+        for l in range(L):
+            kb, vb = pat.buffer_kv(l)
+            assert torch.equal(kb.view(torch.int16), steps[-1][l]["k"].view(torch.int16))
+            assert torch.equal(vb.view(torch.int16), steps[-1][l]["v"].view(torch.int16))
+    finally:
+        pat.close()
