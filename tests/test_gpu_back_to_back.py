@@ -25,16 +25,17 @@ pytestmark = pytest.mark.gpu
 PF, DF = pa.PF_SCHED_PIPEFUSION, pa.PF_SCHED_DISTRIFUSION
 
 
-@pytest.mark.parametrize("d,schedule", [(64, PF), (72, PF), (128, PF), (64, DF), (128, DF)])
-def test_overlapped_micro_steps_match_the_oracle(d, schedule):
-    wl = synth.AttnWorkload("b2b", batch=1, heads=4, head_dim=d, grid_h=64, grid_w=64,
+@pytest.mark.parametrize("d,schedule,B", [(64, PF, 1), (72, PF, 1), (128, PF, 1), (64, DF, 1), (128, DF, 1),
+                                          (72, PF, 2)])
+def test_overlapped_micro_steps_match_the_oracle(d, schedule, B):
+    wl = synth.AttnWorkload("b2b", batch=B, heads=4, head_dim=d, grid_h=64, grid_w=64,
                             n_patches=8, n_txt=77, n_layers=2, n_steps=3, ar_a=0.95, ar_b=0.3)
     S, L, M, P, T = wl.n_steps, wl.n_layers, wl.n_patches, wl.patch_len, wl.n_txt
     gen = synth.AttnInputs(wl, seed=21, device="cuda")
     steps = [[gen.step_tensors(l) for l in range(L)] for _ in range(S)]
     g = torch.Generator(device="cuda").manual_seed(5)
-    q_txt = [torch.randn(1, T, wl.heads, d, device="cuda", generator=g).bfloat16() for _ in range(L)]
-    pat = pa.PatchAttention(1, wl.heads, d, wl.n_img, M, T, L, schedule=schedule)
+    q_txt = [torch.randn(B, T, wl.heads, d, device="cuda", generator=g).bfloat16() for _ in range(L)]
+    pat = pa.PatchAttention(B, wl.heads, d, wl.n_img, M, T, L, schedule=schedule)
     outs, txt_outs = {}, {}
     try:
         for l in range(L):
@@ -59,23 +60,23 @@ def test_overlapped_micro_steps_match_the_oracle(d, schedule):
         for (s, l, p), o in outs.items():
             cur, prev = steps[s][l], steps[max(s - 1, 0)][l]
             rows = sorted(set([0, P - 1] + list(rng.integers(0, P, 6))))
-            h = int(rng.integers(0, wl.heads))
-            take = lambda x: f64(x[0][:, h:h + 1])
+            h, bi = int(rng.integers(0, wl.heads)), int(rng.integers(0, B))
+            take = lambda x: f64(x[bi][:, h:h + 1])
             ref = attention(take(cur["q"]), take(cur["k"]), take(cur["v"]), take(prev["k"]),
                             take(prev["v"]), take(cur["k_txt"]), take(cur["v_txt"]), p, M,
                             wl.softmax_scale, rows=rows)
-            got = f64(o[0][rows][:, h:h + 1])
+            got = f64(o[bi][rows][:, h:h + 1])
             rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
             assert rel <= 5e-3, (s, l, p, rel)
         for (s, l), o in txt_outs.items():
             # after a step's last patch the buffer holds that step's K/V under both schedules
             cur = steps[s][l]
-            h = int(rng.integers(0, wl.heads))
+            h, bi = int(rng.integers(0, wl.heads)), int(rng.integers(0, B))
             rows = sorted(set([0, T - 1] + list(rng.integers(0, T, 6))))
-            take = lambda x: f64(x[0][:, h:h + 1])
+            take = lambda x: f64(x[bi][:, h:h + 1])
             ref = oracle.attend(take(q_txt[l])[rows], np.concatenate([take(cur["k"]), take(cur["k_txt"])]),
                                 np.concatenate([take(cur["v"]), take(cur["v_txt"])]), wl.softmax_scale)
-            got = f64(o[0][rows][:, h:h + 1])
+            got = f64(o[bi][rows][:, h:h + 1])
             rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
             assert rel <= 5e-3, (s, l, "text", rel)
         for l in range(L):
