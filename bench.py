@@ -256,6 +256,15 @@ def n_sms(dev) -> int:
     return torch.cuda.get_device_properties(dev).multi_processor_count
 
 
+# PipeFusion's schedule over one buffer half per layer (the pages' layout) or two (the same
+# rows; the step being written goes to the other half, so consecutive calls on a layer overlap)
+BUFFER_HALVES = 2
+
+
+def pipefusion_schedule(pa):
+    return pa.PF_SCHED_PIPEFUSION_2H if BUFFER_HALVES == 2 else pa.PF_SCHED_PIPEFUSION
+
+
 class StepRunner:
     """One attention workload resident in HBM: per-layer buffers, `n_sets` alternating input
     sets (AR(1) steps) and outputs.  A step = every patch in order x every layer through
@@ -273,7 +282,7 @@ class StepRunner:
         del gen  # drop the fp32 AR(1) state
         torch.cuda.empty_cache()
         self.set_bytes = set_bytes
-        self.pat = pa.PatchAttention(B, H, d, N, M, T, L)
+        self.pat = pa.PatchAttention(B, H, d, N, M, T, L, schedule=pipefusion_schedule(pa))
         for l in range(L):
             self.pat.init_layer(l, self.sets[0][l]["k"], self.sets[0][l]["v"])
         self.outs = [torch.empty(B, N, H, d, dtype=torch.bfloat16, device=dev) for _ in range(L)]
@@ -417,7 +426,7 @@ def sub_record(pa, name, dev, seed, world, peaks, peak_src, min_timed_s=2.0, max
            "flop_per_step": flop_step,
            "config": {"heads": wl.heads, "head_dim": wl.head_dim, "n_img": wl.n_img,
                       "n_patches": wl.n_patches, "patch_len": wl.patch_len, "n_txt": wl.n_txt,
-                      "layers": wl.n_layers},
+                      "layers": wl.n_layers, "buffer_halves": BUFFER_HALVES},
            "l2": f"{r.n_sets} alternating input sets of {r.set_bytes / 1e6:.0f} MB (together > 2x L2)",
            "roofline": attn_roofline(wl, attn, total / 1e3, peaks, peak_src, clk, sms, load_traffic(name)),
            "clocks": clk}
@@ -541,7 +550,7 @@ def run_gpu(args, world, rank, local):
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "batch": wl.batch, "heads": wl.heads, "head_dim": wl.head_dim,
                    "n_img": wl.n_img, "n_patches": M, "patch_len": P, "n_txt": wl.n_txt, "layers": L,
-                   "calls_per_step": M * L, "flop_per_step": flop_step,
+                   "calls_per_step": M * L, "flop_per_step": flop_step, "buffer_halves": BUFFER_HALVES,
                    "cfg_latent": list(CFG_SHAPE[wl.name]), "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (alternating input sets of "
                          f"{(3 * wl.n_img + 2 * wl.n_txt) * wl.heads * wl.head_dim * 2 * L / 1e9:.1f} GB)"},
@@ -735,7 +744,8 @@ def run_profile_calls(args):
     wl = synth.AttnWorkload(wl0.name, wl0.batch, wl0.heads, wl0.head_dim, wl0.grid_h, wl0.grid_w,
                             wl0.n_patches, wl0.n_txt, 1, 2, wl0.ar_a, wl0.ar_b, wl0.qk_rmsnorm)
     t = synth.AttnInputs(wl, device="cuda").step_tensors(0)
-    pat = pa.PatchAttention(wl.batch, wl.heads, wl.head_dim, wl.n_img, wl.n_patches, wl.n_txt, 1)
+    pat = pa.PatchAttention(wl.batch, wl.heads, wl.head_dim, wl.n_img, wl.n_patches, wl.n_txt, 1,
+                            schedule=pipefusion_schedule(pa))
     pat.init_layer(0, t["k"], t["v"])
     P = wl.patch_len
     for p in range(min(args.profile_calls, wl.n_patches)):
@@ -774,6 +784,7 @@ def run_profile_cfg(args):
 
 
 def main():
+    global BUFFER_HALVES
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--profile-calls", type=int, default=0,
                     help="only run the start-up pass and this many micro-steps of one layer (for ncu)")
@@ -782,6 +793,8 @@ def main():
     ap.add_argument("--profile-norm", action="store_true",
                     help="only run two RMS normalisations of a full-spatial Q of the workload (for ncu)")
     ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--buffer-halves", type=int, default=BUFFER_HALVES, choices=[1, 2],
+                    help="PipeFusion over one K/V buffer half per layer or two (same results)")
     ap.add_argument("--steps", type=int, default=12)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="patchattn", choices=["patchattn", "reference"])
@@ -792,6 +805,7 @@ def main():
     ap.add_argument("--no-sub", action="store_true",
                     help="skip the sd3/pixart sub-records (timed over >= 2 s each)")
     args = ap.parse_args()
+    BUFFER_HALVES = args.buffer_halves
     if args.warmup < 3 and args.impl != "reference":
         args.warmup = 3
     if args.profile_calls > 0:

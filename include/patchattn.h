@@ -66,8 +66,18 @@ typedef enum {
  *  PF_SCHED_DISTRIFUSION: every other patch is seen at the previous step (the buffer is
  *    only written after the last patch of the step), the schedule of DistriFusion
  *    ("기술 요약: PipeFusion", 문제 정의: DistriFusion keeps full-spatial stale K/V).
- *    Patches may come in any order, each once per step; the step ends after M calls. */
-typedef enum { PF_SCHED_PIPEFUSION = 0, PF_SCHED_DISTRIFUSION = 1 } pf_schedule;
+ *    Patches may come in any order, each once per step; the step ends after M calls.
+ *  PF_SCHED_PIPEFUSION_2H: the rows PF_SCHED_PIPEFUSION sees, bit for bit, kept in two
+ *    buffer halves: the step being computed writes its patches into one half while the
+ *    previous step's rows stay in the other, and the halves swap after patch M-1.  Twice
+ *    the buffer memory; in exchange a call's scatter never overwrites rows that the
+ *    step's earlier calls are still reading, so consecutive calls on one layer overlap on
+ *    the GPU (with a workspace, see pf_workspace_bytes).  Patches in order, as PIPEFUSION. */
+typedef enum {
+  PF_SCHED_PIPEFUSION = 0,
+  PF_SCHED_DISTRIFUSION = 1,
+  PF_SCHED_PIPEFUSION_2H = 2
+} pf_schedule;
 
 typedef struct {
   int batch;           /* B >= 1 */
@@ -84,9 +94,9 @@ typedef struct {
 typedef struct pf_ctx pf_ctx; /* opaque, host-only */
 
 /* Bytes of ONE layer's K/V buffer: K region [B, N, H, d] bf16 followed by the V region of
- * the same size (2 * B * N * H * d * 2 bytes); under PF_SCHED_DISTRIFUSION a second such
- * [K | V] half follows (the step being written while the other half is read), twice the
- * bytes.  0 if cfg is NULL or invalid. */
+ * the same size (2 * B * N * H * d * 2 bytes); under PF_SCHED_DISTRIFUSION and
+ * PF_SCHED_PIPEFUSION_2H a second such [K | V] half follows (the step being written while
+ * the other half holds the previous step), twice the bytes.  0 if cfg is NULL or invalid. */
 size_t pf_kvbuf_bytes(const pf_config* cfg);
 
 /* Create a context.  kvbuf_per_layer: host array of n_layers device pointers, each to a
@@ -102,7 +112,8 @@ pf_status pf_destroy(pf_ctx* ctx);
 
 /* Start-up pass ("기술 요약: PipeFusion", 핵심 메커니즘 2: stale data exists only after the
  * initial start): copy the first step's full-spatial K and V, [B, N, H, d] bf16 each,
- * into layer `layer`'s buffer and reset that layer's patch counter to 0.  A bit copy. */
+ * into layer `layer`'s buffer (with two halves: into the half pf_get_read_half names) and
+ * reset that layer's patch counter to 0.  A bit copy. */
 pf_status pf_kvbuf_init(pf_ctx* ctx, int layer, const void* k_full, const void* v_full,
                         void* stream);
 
@@ -114,8 +125,9 @@ pf_status pf_kvbuf_init(pf_ctx* ctx, int layer, const void* k_full, const void* 
  *                   k_p, v_p.
  * The call also writes k_p, v_p into the buffer rows of patch p, fused into the attention
  * kernel: under PF_SCHED_PIPEFUSION into the buffer it reads (later patches of the step see
- * them), under PF_SCHED_DISTRIFUSION into the other half, which becomes the half read once
- * all M patches of the step have been called.  o_p must not alias any input.
+ * them), under PF_SCHED_DISTRIFUSION and PF_SCHED_PIPEFUSION_2H into the other half, which
+ * becomes the half read once all M patches of the step have been called (PIPEFUSION_2H reads
+ * the rows of patches < p from that other half).  o_p must not alias any input.
  * Errors: PF_ERR_STATE before pf_kvbuf_init(layer); PF_ERR_ORDER if `patch` is not the
  * layer's next patch (PipeFusion) or was already called this step (DistriFusion);
  * PF_ERR_INVALID_ARG / PF_ERR_ALIGN for bad pointers. */
@@ -127,7 +139,9 @@ pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
  * 주장): the step's text queries attend to the layer's K/V buffer as it stands plus the text
  * keys/values, softmax(scale Q_txt [K_buf;K_txt]^T) [V_buf;V_txt].  Called after the last
  * patch of a step, the buffer holds that step's K/V everywhere.  The buffer is only read
- * and the patch counter is not moved.
+ * and the patch counter is not moved.  "As it stands": under PF_SCHED_PIPEFUSION_2H, the
+ * rows of the step's patches called so far and the previous step's rows of the others;
+ * under PF_SCHED_DISTRIFUSION, the half being read.
  *   q_txt, k_txt, v_txt, o_txt : [B, T, H, d] bf16 (o_txt must not alias an input)
  * Errors: PF_ERR_SHAPE if the configuration has no text tokens; PF_ERR_STATE before
  * pf_kvbuf_init(layer). */
@@ -150,10 +164,11 @@ pf_status pf_qk_rmsnorm(void* x, int64_t n_vectors, int head_dim, const void* ga
  * query tile's key range over several CTAs so that the grid fills the GPU's SMs in near-whole
  * waves; the parts are merged exactly in the log-sum-exp sense (rescaled by their row maxima)
  * by the last part to finish.  The workspace also holds per-layer ordering counters: a call
- * reads a layer's buffer once the earlier calls on that layer have scattered into it, and
- * scatters once they have finished reading it, so consecutive calls on different layers of
- * one stream overlap on the GPU (without a workspace, each call waits for the previous one
- * before it touches the buffer). */
+ * reads a layer's buffer rows once the earlier calls that wrote them have scattered, and
+ * scatters once the earlier calls that read the rows it overwrites have finished reading
+ * (with two buffer halves, the calls up to the previous step's call for the same patch), so
+ * consecutive calls of one stream overlap on the GPU (without a workspace, each call waits
+ * for the previous one before it touches the buffer). */
 size_t pf_workspace_bytes(const pf_config* cfg);
 
 /* Attach a caller-owned device workspace (16-byte aligned, >= pf_workspace_bytes(cfg))
@@ -167,8 +182,16 @@ pf_status pf_set_workspace(pf_ctx* ctx, void* ws, size_t ws_bytes, void* stream)
  * layer's whole state is its buffer contents plus this counter. */
 pf_status pf_get_state(const pf_ctx* ctx, int layer, int* next_patch);
 
-/* Restore a counter saved with pf_get_state (the caller restores the buffer contents). */
+/* Restore a counter saved with pf_get_state (the caller restores the buffer contents).
+ * Under the two-half schedules only the start of a step (next_patch 0) can be restored
+ * (else PF_ERR_UNSUPPORTED); the caller restores the half pf_get_read_half names. */
 pf_status pf_set_state(pf_ctx* ctx, int layer, int next_patch);
+
+/* Which half of the layer's buffer holds the previous step's rows (the half read for the
+ * patches not yet called in this step): 0 or 1 under PF_SCHED_DISTRIFUSION and
+ * PF_SCHED_PIPEFUSION_2H, where the halves swap after each step's last patch; always 0
+ * under PF_SCHED_PIPEFUSION.  Errors: PF_ERR_INVALID_ARG for a bad layer or pointer. */
+pf_status pf_get_read_half(const pf_ctx* ctx, int layer, int* half);
 
 /* Workspace bytes pf_cfg_combine_relmae needs for `batch` samples of `n_per_sample`
  * floats (0 on invalid sizes). */

@@ -31,13 +31,14 @@ PF_ERR_TIMEOUT = 8
 
 PF_SCHED_PIPEFUSION = 0
 PF_SCHED_DISTRIFUSION = 1
+PF_SCHED_PIPEFUSION_2H = 2
 
 EXPORTED = [
     "pf_kvbuf_bytes", "pf_create", "pf_destroy", "pf_kvbuf_init", "pf_patch_attn_step",
     "pf_get_state", "pf_set_state", "pf_workspace_bytes", "pf_set_workspace",
     "pf_cfg_workspace_bytes", "pf_cfg_combine_relmae", "pf_cfg_combine_relmae_static",
     "pf_check_device_status", "pf_selftest_bounded_wait", "pf_status_string", "pf_version", "pf_switch_init",
-    "pf_switch_update", "pf_text_attn_step", "pf_qk_rmsnorm",
+    "pf_switch_update", "pf_text_attn_step", "pf_qk_rmsnorm", "pf_get_read_half",
 ]
 
 PF_PHASE_WARMUP = 0
@@ -87,6 +88,7 @@ def _lib():
             "pf_kvbuf_init": (i, [vp, i, vp, vp, vp]),
             "pf_patch_attn_step": (i, [vp, i, i, vp, vp, vp, vp, vp, vp, vp]),
             "pf_get_state": (i, [vp, i, ctypes.POINTER(i)]),
+            "pf_get_read_half": (i, [vp, i, ctypes.POINTER(i)]),
             "pf_workspace_bytes": (sz, [cfgp]),
             "pf_set_workspace": (i, [vp, vp, sz, vp]),
             "pf_set_state": (i, [vp, i, i]),
@@ -230,6 +232,12 @@ def pf_set_state(ctx, layer: int, next_patch: int) -> None:
     _check(_lib().pf_set_state(ctx, layer, next_patch), "pf_set_state")
 
 
+def pf_get_read_half(ctx, layer: int) -> int:
+    v = ctypes.c_int()
+    _check(_lib().pf_get_read_half(ctx, layer, ctypes.byref(v)), "pf_get_read_half")
+    return v.value
+
+
 def pf_cfg_workspace_bytes(batch: int, n_per_sample: int) -> int:
     return int(_lib().pf_cfg_workspace_bytes(batch, n_per_sample))
 
@@ -307,7 +315,7 @@ class PatchAttention:
     """A context plus its per-layer K/V buffers, allocated by torch on ``device``.
 
     Buffer layout per layer (uint8 tensor): K [B, N, H, d] bf16 then V of the same size
-    (DistriFusion schedule: two such halves).
+    (DistriFusion and two-half PipeFusion schedules: two such halves).
     """
 
     def __init__(self, batch, heads, head_dim, n_img, n_patches, n_txt, n_layers,
@@ -359,6 +367,22 @@ class PatchAttention:
 
     def next_patch(self, layer):
         return pf_get_state(self.ctx, layer)
+
+    def read_half(self, layer):
+        return pf_get_read_half(self.ctx, layer)
+
+    def buffer_as_it_stands(self, layer):
+        """(K, V) copies of the rows a text-token call on the layer would see now: under the
+        two-half PipeFusion schedule the step's patches called so far come from the half being
+        written and the other rows from the half being read; otherwise the half being read."""
+        rd = self.read_half(layer)
+        k, v = (t.clone() for t in self.buffer_kv(layer, rd))
+        if self.cfg.schedule == PF_SCHED_PIPEFUSION_2H:
+            n = self.next_patch(layer) * self.plen
+            kw, vw = self.buffer_kv(layer, 1 - rd)
+            k[:, :n] = kw[:, :n]
+            v[:, :n] = vw[:, :n]
+        return k, v
 
     def check(self, stream=None):
         pf_check_device_status(self.ctx, stream)

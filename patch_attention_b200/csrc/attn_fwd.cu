@@ -22,9 +22,11 @@
 // accumulates in TMEM.
 // The context is walked as segments so that patch p's rows are read from the fresh
 // tensors, never from buffer rows that other CTAs of this launch are writing:
-//   [fresh rows 0..P) | buffer rows 0..pP) | buffer rows (p+1)P..N) | text rows 0..T)
-// Softmax is permutation invariant over keys, so this order gives the same result as
-// the natural token order.  Row maxima are kept lazily: O is rescaled only when a row's
+//   [fresh rows 0..P) | text rows 0..T) | buffer rows (p+1)P..N) | buffer rows 0..pP)
+// The call's own tensors come first and the rows that the step's earlier calls wrote
+// come last, so a launch has the most work it can do before those calls' writes must be
+// complete.  Softmax is permutation invariant over keys, so this order gives the same
+// result as the natural token order.  Row maxima are kept lazily: O is rescaled only when a row's
 // maximum grows by more than 2^8, which is exact because the final O / l uses the same
 // reference maximum for numerator and denominator.
 //
@@ -37,8 +39,16 @@
 // in part order, O = sum_i 2^(m_i - M) O_i / sum_i 2^(m_i - M) l_i, into the bf16 output.
 //
 // Ordering between launches: with a workspace, calls on one layer buffer are ordered by two
-// per-layer counters (CTAs that finished their scatter, CTAs that finished reading the
-// buffer) instead of by the completion of the previous grid, so that launches overlap.
+// per-layer counters in global memory instead of by the completion of the previous grid, so
+// that launches overlap: CTAs that finished their scatter share and CTAs that finished
+// reading the buffer, each counted in call order, so that a counter reaching the host's total
+// for a prefix of the calls means that prefix is done.  Before its buffer rows a launch waits
+// for the scatters of the calls that wrote them; a scatter waits for the reads of the calls
+// that read the rows it overwrites.  With a single buffer half those are all earlier calls.
+// With two halves (the step being written goes to the other half) the rows of patch p in the
+// half being written were last read by the calls before patch p of the previous step, so
+// consecutive calls of a step wait on each other only where a call reads rows that the
+// step's earlier calls wrote (its lo rows, walked last).
 //
 // Every wait is bounded (2 s); on expiry the kernel records the role in a device word,
 // raises a CTA-wide abort flag, drains its in-flight copies and MMAs, frees TMEM and
@@ -162,24 +172,34 @@ struct Segments {
     n_txt = (txt_len + kRows - 1) / kRows;
   }
   __device__ int total() const { return n_fresh + n_lo + n_hi + n_txt; }
-  // src: 0 = fresh tensors, 1 = buffer rows [0, lo_len) through the maps bounded at lo_len
-  // (a ragged last tile reads zeros past the segment, never the rows of patch p that the
-  // scatter of this launch is writing), 2 = text, 3 = buffer rows from hi_row0 (bounded by
-  // the end of the buffer)
+  // Segment k in walk order (fresh, text, hi, lo): its last tile index + 1 and its rows.
+  __device__ void bounds(int k, int& end, int& len) const {
+    const int n[4] = {n_fresh, n_txt, n_hi, n_lo};
+    const int r[4] = {plen, txt_len, hi_len, lo_len};
+    end = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (i <= k) end += n[i];
+    len = r[k];
+  }
+  // src: 0 = fresh tensors, 2 = text, 3 = buffer rows from hi_row0 (bounded by the end of
+  // the buffer), 1 = buffer rows [0, lo_len) through the maps bounded at lo_len (a ragged
+  // last tile reads zeros past the segment, never the rows of patch p that the scatter of
+  // this launch is writing)
   __device__ void tile(int j, int& src, int& row0, int& nvalid) const {
     if (j < n_fresh) {
       src = 0; row0 = j * kRows; nvalid = min(kRows, plen - row0); return;
     }
     j -= n_fresh;
-    if (j < n_lo) {
-      src = 1; row0 = j * kRows; nvalid = min(kRows, lo_len - row0); return;
+    if (j < n_txt) {
+      src = 2; row0 = j * kRows; nvalid = min(kRows, txt_len - row0); return;
     }
-    j -= n_lo;
+    j -= n_txt;
     if (j < n_hi) {
       src = 3; row0 = hi_row0 + j * kRows; nvalid = min(kRows, hi_len - j * kRows); return;
     }
     j -= n_hi;
-    src = 2; row0 = j * kRows; nvalid = min(kRows, txt_len - row0);
+    src = 1; row0 = j * kRows; nvalid = min(kRows, lo_len - row0);
   }
 };
 
@@ -346,10 +366,12 @@ __device__ __forceinline__ void raise_abort(volatile int* abort, unsigned code) 
 template <int D>
 __device__ __forceinline__ void scatter_share(const AttnParams& p, int lane) {
   if (p.k_dst == nullptr) return;
-  // earlier calls on the layer read these buffer rows (as stale context): wait until every
-  // CTA of theirs has finished reading (or, without counters, for the previous grid)
-  if (p.dep_read != nullptr) {
-    if (!wait_count_geq64(p.dep_read, p.dep_read_target, nullptr, kWaitNs)) {
+  // scatters go in call order, and earlier calls read these buffer rows: wait until every
+  // earlier scatter is done and every CTA of those calls has finished reading (or, without
+  // counters, for the previous grid)
+  if (p.dep_scat != nullptr) {
+    if (!wait_count_geq64(p.dep_scat, p.dep_scat_target, nullptr, kWaitNs) ||
+        !wait_count_geq64(p.dep_read, p.dep_war_target, nullptr, kWaitNs)) {
       if (lane == 0) atomicOr(&g_watchdog, kWdScatter);
       return;
     }
@@ -394,6 +416,40 @@ __device__ __forceinline__ void scatter_share(const AttnParams& p, int lane) {
     __syncwarp();
     if (lane == 0) count_release(p.dep_scat);
   }
+}
+
+// The producer's wait before its first tile of buffer rows of one kind: hi rows (src 3) were
+// written by calls of earlier epochs, lo rows (src 1) by earlier calls that may belong to
+// this epoch.  Without counters, one wait for the previous grid covers both.  False when a
+// bounded wait gave up.
+__device__ __forceinline__ bool buffer_rows_ready(const AttnParams& p, int src, bool& hi_done,
+                                                  bool& lo_done, const volatile int* abort) {
+  if (p.dep_scat == nullptr) {
+    if (!hi_done && !lo_done) grid_dep_wait();
+    hi_done = lo_done = true;
+    return true;
+  }
+  if (src == 3 && !hi_done) {
+    if (!wait_count_geq64(p.dep_scat, p.dep_hi_target, abort, kWaitNs)) return false;
+    hi_done = true;
+  }
+  if (src == 1 && !lo_done) {
+    if (!wait_count_geq64(p.dep_scat, p.dep_lo_target, abort, kWaitNs)) return false;
+    lo_done = true;
+  }
+  return true;
+}
+
+// Count this CTA's finished reads (after its copies have landed), once every CTA of the
+// layer's earlier calls has counted its own: the counter then passes the total of a prefix of
+// the calls only when exactly that prefix has finished reading.
+__device__ __forceinline__ void count_reads_done(const AttnParams& p) {
+  if (p.dep_read == nullptr) return;
+  if (!wait_count_geq64(p.dep_read, p.dep_read_target, nullptr, kWaitNs)) {
+    atomicOr(&g_watchdog, kWdLoad);
+    return;
+  }
+  count_release(p.dep_read);
 }
 
 // After the merge, the partial slots of a query tile ([part][d + 2][128] fp32) are dead: the next launch writes every slot before it reads one.  Dropping their L2 lines
@@ -618,22 +674,13 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
           tma_load_4d(smem_u32(sQ + t * kHrTile), &p.tm_q, 0, hd, q0 + t * kRows, b, qbar);
         int issued = 0;
         bool ok = true;
-        bool dep_done = false;
+        bool dep_hi = false, dep_lo = false;
         for (int j = 0; j < n_tiles && ok; ++j) {
           int src, row0, nv;
           seg.tile(j0 + j, src, row0, nv);
-          if ((src == 1 || src == 3) && !dep_done) {
-            // buffer rows: wait until every earlier call on the layer has scattered into the
-            // buffer (or, without counters, for the previous grid)
-            if (p.dep_scat != nullptr) {
-              if (!wait_count_geq64(p.dep_scat, p.dep_scat_target, abort, kWaitNs)) {
-                ok = false;
-                break;
-              }
-            } else {
-              grid_dep_wait();
-            }
-            dep_done = true;
+          if ((src == 1 || src == 3) && !buffer_rows_ready(p, src, dep_hi, dep_lo, abort)) {
+            ok = false;
+            break;
           }
           for (int kv = 0; kv < 2; ++kv) {
             const int i = 2 * j + kv;
@@ -658,7 +705,7 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
         for (int i = issued > S ? issued - S : 0; i < issued; ++i)
           mbar_wait(smem_u32(kv_full + (i % S)), (i / S) & 1, nullptr, kWaitNs);
         // this CTA has read all it reads of the buffer: count it for later calls' scatters
-        if (p.dep_read != nullptr) count_release(p.dep_read);
+        count_reads_done(p);
       }
     } else if (warp == kHrWarpMma0 || (NQ == 2 && warp == kHrWarpMma1)) {
       // ------------------------------------------------------------ MMA issuer of query tile t
@@ -747,13 +794,12 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
     // local indices of this CTA's ragged context tiles and the valid keys of this half there
     int rag_j[4], rag_nv[4];
     {
-      const int ends[4] = {seg.n_fresh, seg.n_fresh + seg.n_lo, seg.n_fresh + seg.n_lo + seg.n_hi,
-                           seg.total()};
-      const int lens[4] = {seg.plen, seg.lo_len, seg.hi_len, seg.txt_len};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const int e = ends[k] - 1;
-        const int nv = lens[k] % kRows;
+        int end, len;
+        seg.bounds(k, end, len);
+        const int e = end - 1;
+        const int nv = len % kRows;
         rag_nv[k] = min(max(nv - 64 * hh, 0), 64);
         rag_j[k] = (nv != 0 && e >= j0 && e < j1) ? e - j0 : -1;
       }
@@ -1223,22 +1269,13 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
                         q0 + t * kRows, b, qbar);
         int issued = 0;
         bool ok = true;
-        bool dep_done = false;
+        bool dep_hi = false, dep_lo = false;
         for (int j = 0; j < n_tiles && ok; ++j) {
           int src, row0, nv;
           seg.tile(j0 + j, src, row0, nv);
-          if ((src == 1 || src == 3) && !dep_done) {
-            // buffer rows: wait until every earlier call on the layer has scattered into the
-            // buffer (or, without counters, for the previous grid)
-            if (p.dep_scat != nullptr) {
-              if (!wait_count_geq64(p.dep_scat, p.dep_scat_target, abort, kWaitNs)) {
-                ok = false;
-                break;
-              }
-            } else {
-              grid_dep_wait();
-            }
-            dep_done = true;
+          if ((src == 1 || src == 3) && !buffer_rows_ready(p, src, dep_hi, dep_lo, abort)) {
+            ok = false;
+            break;
           }
           for (int kv = 0; kv < 2; ++kv) {
             const int i = 2 * j + kv;
@@ -1265,7 +1302,7 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
         for (int i = issued > S ? issued - S : 0; i < issued; ++i)
           mbar_wait(smem_u32(kv_full + (i % S)), (i / S) & 1, nullptr, kWaitNs);
         // this CTA has read all it reads of the buffer: count it for later calls' scatters
-        if (p.dep_read != nullptr) count_release(p.dep_read);
+        count_reads_done(p);
       }
     } else if (warp == kWarpMma || (NQ == 2 && warp == kWarpMma2)) {
       // ------------------------------------------------------------ MMA issuer of query tile t
@@ -1358,13 +1395,12 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
     // local indices of this CTA's ragged context tiles and their valid rows
     int rag_j[4], rag_nv[4];
     {
-      const int ends[4] = {seg.n_fresh, seg.n_fresh + seg.n_lo, seg.n_fresh + seg.n_lo + seg.n_hi,
-                           seg.total()};
-      const int lens[4] = {seg.plen, seg.lo_len, seg.hi_len, seg.txt_len};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const int e = ends[k] - 1;
-        rag_nv[k] = lens[k] % kRows;
+        int end, len;
+        seg.bounds(k, end, len);
+        const int e = end - 1;
+        rag_nv[k] = len % kRows;
         rag_j[k] = (rag_nv[k] != 0 && e >= j0 && e < j1) ? e - j0 : -1;
       }
     }
@@ -1513,10 +1549,12 @@ int attn_choose_split(int n_pairs, int n_tiles, int n_sms, int max_split) {
   // Cost model in units of context tiles.  Launches overlap on the GPU (the per-layer ordering
   // counters let a launch start while earlier ones finish), so a call costs the larger of its
   // share of SM time, n_pairs (n_tiles + k c) / n_sms, and half the length of one CTA,
-  // (ceil(n_tiles / k) + c) / 2: at most two launches on one layer buffer make progress at
-  // once (the next one reads after this one's scatter, scatters after this one's reads).  c is
-  // the fixed cost of a CTA (launch, TMEM allocation, Q load, pipeline fill, merge).  Of the
-  // splits within 5% of the cheapest the smallest is taken: fewer partials to store and merge.
+  // (ceil(n_tiles / k) + c) / 2: a launch is issued only once every CTA of the previous one
+  // has started, so short launches of few CTAs leave SMs idle between them (measured: a
+  // PixArt-size call of 32 CTAs runs 8-12% slower unsplit than split in two, with either
+  // buffer layout).  c is the fixed cost of a CTA (launch, TMEM allocation, Q load, pipeline
+  // fill, merge).  Of the splits within 5% of the cheapest the smallest is taken: fewer
+  // partials to store and merge.
   constexpr double kOverheadTiles = 6.0;
   const int kmax = max_split < kMaxSplit ? max_split : kMaxSplit;
   double cost[kMaxSplit + 1];

@@ -24,16 +24,21 @@ struct pf_ctx {
   std::vector<uint8_t*> base;    // per layer, caller-owned
   std::vector<int> next_patch;   // PipeFusion: the patch the layer expects next
   std::vector<int> initialised;
-  std::vector<int> read_half;    // DistriFusion: which half of the buffer holds the stale step
+  std::vector<int> read_half;    // two halves: which half holds the previous step's rows
   std::vector<std::vector<uint8_t>> seen;  // DistriFusion: patches done in the current step
   std::vector<int> seen_count;
   uint8_t* ws = nullptr;         // optional attention workspace (caller-owned)
   size_t ws_bytes = 0;
   int n_sms = 0;                 // queried on first use
-  // per layer: the CTAs of the calls launched so far that will count a finished scatter /
-  // finished buffer reads on the workspace's ordering counters (reset with the workspace)
+  // Per layer, for the workspace's ordering counters (reset with the workspace): the CTAs of
+  // the calls launched so far that will count a finished scatter, and those that will count
+  // finished reads; both as they stood when the current step began; and, per patch, the read
+  // count just before that patch's call of the previous step (two buffer halves).
   std::vector<unsigned long long> scat_target;
   std::vector<unsigned long long> read_target;
+  std::vector<unsigned long long> scat_step_start;
+  std::vector<unsigned long long> read_step_start;
+  std::vector<std::vector<unsigned long long>> read_before_patch;
 };
 
 namespace {
@@ -67,7 +72,8 @@ pf_status check_config(const pf_config* c) {
     return PF_ERR_SHAPE;
   if (c->n_img % c->n_patches != 0) return PF_ERR_SHAPE;
   if (c->head_dim != 64 && c->head_dim != 72 && c->head_dim != 128) return PF_ERR_UNSUPPORTED;
-  if (c->schedule != PF_SCHED_PIPEFUSION && c->schedule != PF_SCHED_DISTRIFUSION)
+  if (c->schedule != PF_SCHED_PIPEFUSION && c->schedule != PF_SCHED_DISTRIFUSION &&
+      c->schedule != PF_SCHED_PIPEFUSION_2H)
     return PF_ERR_UNSUPPORTED;
   if (!(c->softmax_scale >= 0.f) || std::isinf(c->softmax_scale)) return PF_ERR_INVALID_ARG;
   // TMA coordinates and per-row offsets are 32-bit
@@ -126,14 +132,19 @@ constexpr int kAssumedSms = 148;
 
 // Counters first (fixed place, sized for the larger of patch and text-query calls), then the
 // partial slots.
-// Two counters (parts arrived, partials written) per query tile of every pair, then two 64-bit
-// ordering counters (CTAs that finished their scatter, CTAs that finished reading the buffer)
-// per layer.
+// Two counters (parts arrived, partials written) per query tile of every pair, then two
+// 64-bit ordering counters per layer (CTAs that finished their scatter, CTAs that finished
+// reading the buffer).
 size_t pair_counter_bytes(int pairs) { return static_cast<size_t>(pairs) * 2 * 2 * 4; }
 size_t counter_bytes(const pf_config& c) {
   const size_t b = pair_counter_bytes(pairs_of(c)) + static_cast<size_t>(c.n_layers) * 2 * 8;
   return ((b + 255) / 256) * 256;
 }
+
+// A layer with two buffer halves: the step being written goes to the half that the step does
+// not read (DistriFusion, and PipeFusion over two halves).
+bool two_halves(const pf_config& c) { return c.schedule != PF_SCHED_PIPEFUSION; }
+
 
 size_t workspace_for(const pf_config& c, int n_sms) {
   const int plen = c.n_img / c.n_patches;
@@ -155,9 +166,27 @@ size_t workspace_for(const pf_config& c, int n_sms) {
 
 bool layer_ok(const pf_ctx* ctx, int layer) { return layer >= 0 && layer < ctx->cfg.n_layers; }
 
+// A step of a layer starts (two buffer halves): record the counts its calls' waits refer to.
+// After pf_kvbuf_init or pf_set_state every earlier call has finished (the start-up copy
+// waits for the stream's earlier work), so the previous step's per-patch counts are dropped.
+void begin_step(pf_ctx* ctx, int layer, bool restart) {
+  if (ctx->ws == nullptr) return;
+  ctx->scat_step_start[layer] = ctx->scat_target[layer];
+  ctx->read_step_start[layer] = ctx->read_target[layer];
+  if (restart)
+    std::fill(ctx->read_before_patch[layer].begin(), ctx->read_before_patch[layer].end(),
+              ctx->read_target[layer]);
+}
+
+// What a call on a layer waits for, as counts of the layer's ordering counters.
+struct Waits {
+  unsigned long long hi, lo, war;  // scatters before hi rows / lo rows; reads before the scatter
+};
+
 // Fill the fields common to every attention call (sizes, scale, work decomposition and
-// key-range split) and launch.  p carries the tensor maps, pointers and segments.
-cudaError_t launch_attention(pf_ctx* ctx, pf::AttnParams& p, int layer, void* stream) {
+// key-range split) and launch.  p carries the tensor maps, pointers and segments; w what the
+// call waits for (with a workspace).
+cudaError_t launch_attention(pf_ctx* ctx, pf::AttnParams& p, int layer, const Waits& w, void* stream) {
   const pf_config& c = ctx->cfg;
   p.batch = c.batch;
   p.heads = c.heads;
@@ -200,7 +229,10 @@ cudaError_t launch_attention(pf_ctx* ctx, pf::AttnParams& p, int layer, void* st
         ctx->ws + pair_counter_bytes(pairs_of(c))) + static_cast<size_t>(layer) * 2;
     p.dep_scat = dep;
     p.dep_read = dep + 1;
+    p.dep_hi_target = w.hi;
+    p.dep_lo_target = w.lo;
     p.dep_scat_target = ctx->scat_target[layer];
+    p.dep_war_target = w.war;
     p.dep_read_target = ctx->read_target[layer];
   }
   const cudaError_t e = pf::launch_patch_attn(p, static_cast<cudaStream_t>(stream));
@@ -213,7 +245,7 @@ cudaError_t launch_attention(pf_ctx* ctx, pf::AttnParams& p, int layer, void* st
   return e;
 }
 
-// K/V regions of a layer's buffer: half 0 is [K | V]; DistriFusion adds half 1 [K | V].
+// K/V regions of a layer's buffer: half 0 is [K | V]; two-half schedules add half 1 [K | V].
 uint8_t* region(const pf_ctx* ctx, int layer, int half, int kv) {
   const size_t bytes = ctx->tensor_elems * 2;
   return ctx->base[layer] + (static_cast<size_t>(half) * 2 + kv) * bytes;
@@ -241,7 +273,7 @@ extern "C" {
 
 size_t pf_kvbuf_bytes(const pf_config* cfg) {
   if (check_config(cfg) != PF_OK) return 0;
-  const size_t halves = cfg->schedule == PF_SCHED_DISTRIFUSION ? 2 : 1;
+  const size_t halves = two_halves(*cfg) ? 2 : 1;
   return halves * 2 * region_elems(cfg) * 2;
 }
 
@@ -296,6 +328,7 @@ pf_status pf_kvbuf_init(pf_ctx* ctx, int layer, const void* k_full, const void* 
   ctx->next_patch[layer] = 0;
   std::fill(ctx->seen[layer].begin(), ctx->seen[layer].end(), 0);
   ctx->seen_count[layer] = 0;
+  begin_step(ctx, layer, true);
   return PF_OK;
 }
 
@@ -312,8 +345,9 @@ pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
       (k_txt && !aligned16(k_txt)) || (v_txt && !aligned16(v_txt)))
     return PF_ERR_ALIGN;
   if (!ctx->initialised[layer]) return PF_ERR_STATE;
-  const bool pipefusion = c.schedule == PF_SCHED_PIPEFUSION;
-  if (pipefusion) {
+  // PipeFusion (either buffer layout) takes the patches in order; DistriFusion in any order
+  const bool in_order = c.schedule != PF_SCHED_DISTRIFUSION;
+  if (in_order) {
     if (patch != ctx->next_patch[layer]) return PF_ERR_ORDER;
   } else {
     if (ctx->seen[layer][patch]) return PF_ERR_ORDER;
@@ -324,7 +358,11 @@ pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
   pf::AttnParams p;
   std::memset(&p, 0, sizeof(p));
   const int read = ctx->read_half[layer];
-  const int write = pipefusion ? read : 1 - read;
+  const int write = two_halves(c) ? 1 - read : read;
+  // rows of patches < p: this step's (PipeFusion) are in the half being written; the previous
+  // step's (DistriFusion) in the half being read
+  const bool lo_current = c.schedule != PF_SCHED_DISTRIFUSION;
+  const int lo_half = lo_current ? write : read;
   const int lo_len = patch * plen;
   if (!make_map(&p.tm_q, q_p, c.batch, plen, c.heads, d) ||
       !make_map(&p.tm_kf, k_p, c.batch, plen, c.heads, d) ||
@@ -335,8 +373,8 @@ pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
   // the rows before the patch through maps that end at the patch: the last tile of that
   // segment reads zeros, not the patch's own rows, which this launch's scatter is writing
   if (lo_len > 0 &&
-      (!make_map(&p.tm_kl, region(ctx, layer, read, 0), c.batch, lo_len, c.heads, d, c.n_img) ||
-       !make_map(&p.tm_vl, region(ctx, layer, read, 1), c.batch, lo_len, c.heads, d, c.n_img)))
+      (!make_map(&p.tm_kl, region(ctx, layer, lo_half, 0), c.batch, lo_len, c.heads, d, c.n_img) ||
+       !make_map(&p.tm_vl, region(ctx, layer, lo_half, 1), c.batch, lo_len, c.heads, d, c.n_img)))
     return PF_ERR_CUDA;
   if (c.n_txt > 0 && (!make_map(&p.tm_kt, k_txt, c.batch, c.n_txt, c.heads, d) ||
                       !make_map(&p.tm_vt, v_txt, c.batch, c.n_txt, c.heads, d)))
@@ -353,21 +391,47 @@ pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
   p.lo_len = lo_len;
   p.hi_row0 = (patch + 1) * plen;
   p.hi_len = c.n_img - (patch + 1) * plen;
-  const pf_status ls = from_attn_launch(launch_attention(ctx, p, layer, stream));
+  Waits w{};
+  unsigned long long read_before = 0;
+  if (ctx->ws != nullptr) {
+    const unsigned long long all_scat = ctx->scat_target[layer], all_read = ctx->read_target[layer];
+    read_before = all_read;
+    if (c.schedule == PF_SCHED_PIPEFUSION) {
+      // one half: every earlier call wrote rows this call reads or read rows it overwrites
+      w = {all_scat, all_scat, all_read};
+    } else if (c.schedule == PF_SCHED_PIPEFUSION_2H) {
+      // hi rows: written in earlier steps; lo rows: by this step's earlier calls; the rows
+      // of patch p in the half being written: read by the calls before patch p of the
+      // previous step (as its stale rows) and by older ones
+      w = {ctx->scat_step_start[layer], all_scat, ctx->read_before_patch[layer][patch]};
+    } else {
+      // DistriFusion: every row read was written in earlier steps; every call of the
+      // previous step read the rows of the half being written
+      w = {ctx->scat_step_start[layer], ctx->scat_step_start[layer], ctx->read_step_start[layer]};
+    }
+  }
+  const pf_status ls = from_attn_launch(launch_attention(ctx, p, layer, w, stream));
   if (ls != PF_OK) return ls;
+  if (ctx->ws != nullptr) ctx->read_before_patch[layer][patch] = read_before;
 
-  if (pipefusion) {
+  bool step_done = false;
+  if (in_order) {
     ctx->next_patch[layer] = (patch + 1) % c.n_patches;
+    step_done = ctx->next_patch[layer] == 0;
   } else {
     ctx->seen[layer][patch] = 1;
     if (++ctx->seen_count[layer] == c.n_patches) {
-      // every patch of the step wrote its fresh rows into the other half: it becomes the
-      // stale context of the next step
-      ctx->read_half[layer] = 1 - ctx->read_half[layer];
       std::fill(ctx->seen[layer].begin(), ctx->seen[layer].end(), 0);
       ctx->seen_count[layer] = 0;
+      step_done = true;
     }
     ctx->next_patch[layer] = ctx->seen_count[layer];
+  }
+  if (step_done && two_halves(c)) {
+    // every patch of the step wrote its fresh rows into the other half: it becomes the
+    // previous step's half of the next step
+    ctx->read_half[layer] = 1 - ctx->read_half[layer];
+    begin_step(ctx, layer, false);
   }
   return PF_OK;
 }
@@ -384,22 +448,42 @@ pf_status pf_text_attn_step(pf_ctx* ctx, int layer, const void* q_txt, const voi
   if (!ctx->initialised[layer]) return PF_ERR_STATE;
   const int d = c.head_dim;
   const int read = ctx->read_half[layer];
+  const int plen = c.n_img / c.n_patches;
+  // the buffer as it stands: with PipeFusion over two halves, the rows of the patches done in
+  // this step are in the half being written and the rest in the other; otherwise all of it is
+  // in the half being read
+  const bool split_halves = c.schedule == PF_SCHED_PIPEFUSION_2H;
+  const int lo_len = split_halves ? ctx->next_patch[layer] * plen : c.n_img;
   pf::AttnParams p;
   std::memset(&p, 0, sizeof(p));
+  const int lo_half = split_halves ? 1 - read : read;
   if (!make_map(&p.tm_q, q_txt, c.batch, c.n_txt, c.heads, d) ||
-      !make_map(&p.tm_kl, region(ctx, layer, read, 0), c.batch, c.n_img, c.heads, d) ||
-      !make_map(&p.tm_vl, region(ctx, layer, read, 1), c.batch, c.n_img, c.heads, d) ||
       !make_map(&p.tm_kt, k_txt, c.batch, c.n_txt, c.heads, d) ||
       !make_map(&p.tm_vt, v_txt, c.batch, c.n_txt, c.heads, d))
     return PF_ERR_CUDA;
+  if (lo_len > 0 &&
+      (!make_map(&p.tm_kl, region(ctx, layer, lo_half, 0), c.batch, lo_len, c.heads, d, c.n_img) ||
+       !make_map(&p.tm_vl, region(ctx, layer, lo_half, 1), c.batch, lo_len, c.heads, d, c.n_img)))
+    return PF_ERR_CUDA;
+  if (lo_len < c.n_img &&
+      (!make_map(&p.tm_kb, region(ctx, layer, read, 0), c.batch, c.n_img, c.heads, d) ||
+       !make_map(&p.tm_vb, region(ctx, layer, read, 1), c.batch, c.n_img, c.heads, d)))
+    return PF_ERR_CUDA;
   p.o = static_cast<uint16_t*>(o_txt);
-  p.plen = c.n_img / c.n_patches;
+  p.plen = plen;
   p.q_rows = c.n_txt;   // text queries
   p.fresh_rows = 0;     // no fresh patch rows, no scatter (k_dst stays null)
-  p.lo_len = c.n_img;   // the whole buffer as it stands
-  p.hi_row0 = c.n_img;
-  p.hi_len = 0;
-  const pf_status ls = from_attn_launch(launch_attention(ctx, p, layer, stream));
+  p.lo_len = lo_len;
+  p.hi_row0 = lo_len;
+  p.hi_len = c.n_img - lo_len;
+  Waits w{};
+  if (ctx->ws != nullptr) {
+    // lo rows: the half being written (two-half PipeFusion) or the one half; hi rows and
+    // DistriFusion's rows: written in earlier steps
+    const unsigned long long start = two_halves(c) ? ctx->scat_step_start[layer] : ctx->scat_target[layer];
+    w = {start, c.schedule == PF_SCHED_DISTRIFUSION ? start : ctx->scat_target[layer], 0ull};
+  }
+  const pf_status ls = from_attn_launch(launch_attention(ctx, p, layer, w, stream));
   if (ls != PF_OK) return ls;
   return PF_OK;
 }
@@ -421,12 +505,24 @@ pf_status pf_get_state(const pf_ctx* ctx, int layer, int* next_patch) {
   return PF_OK;
 }
 
+pf_status pf_get_read_half(const pf_ctx* ctx, int layer, int* half) {
+  if (!ctx || !half || !layer_ok(ctx, layer)) return PF_ERR_INVALID_ARG;
+  *half = ctx->read_half[layer];
+  return PF_OK;
+}
+
 pf_status pf_set_state(pf_ctx* ctx, int layer, int next_patch) {
   if (!ctx || !layer_ok(ctx, layer)) return PF_ERR_INVALID_ARG;
   if (next_patch < 0 || next_patch >= ctx->cfg.n_patches) return PF_ERR_INVALID_ARG;
   if (ctx->cfg.schedule != PF_SCHED_PIPEFUSION && next_patch != 0) return PF_ERR_UNSUPPORTED;
   ctx->next_patch[layer] = next_patch;
   ctx->initialised[layer] = 1;
+  if (two_halves(ctx->cfg)) {
+    // a step starts
+    std::fill(ctx->seen[layer].begin(), ctx->seen[layer].end(), 0);
+    ctx->seen_count[layer] = 0;
+  }
+  begin_step(ctx, layer, true);
   return PF_OK;
 }
 
@@ -449,8 +545,12 @@ pf_status pf_set_workspace(pf_ctx* ctx, void* ws, size_t ws_bytes, void* stream)
   if (e != cudaSuccess) return PF_ERR_CUDA;
   ctx->ws = static_cast<uint8_t*>(ws);
   ctx->ws_bytes = ws_bytes;
-  ctx->scat_target.assign(ctx->cfg.n_layers, 0ull);
-  ctx->read_target.assign(ctx->cfg.n_layers, 0ull);
+  const int L = ctx->cfg.n_layers;
+  ctx->scat_target.assign(L, 0ull);
+  ctx->read_target.assign(L, 0ull);
+  ctx->scat_step_start.assign(L, 0ull);
+  ctx->read_step_start.assign(L, 0ull);
+  ctx->read_before_patch.assign(L, std::vector<unsigned long long>(ctx->cfg.n_patches, 0ull));
   return PF_OK;
 }
 

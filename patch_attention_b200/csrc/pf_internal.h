@@ -44,15 +44,22 @@ struct AttnParams {
   unsigned* ws_cnt;     // per [pair][tile]: parts arrived, partials written; zero between launches
   int discard;          // drop the merged partials from L2 (1) rather than let them be written back
   // Order against the other calls on the same layer buffer without waiting for the whole
-  // previous grid: the buffer is read once *dep_scat (CTAs of earlier calls on the layer that
-  // finished their scatter) reaches dep_scat_target, and the scatter writes once *dep_read
-  // (CTAs of earlier calls on the layer that finished reading the buffer) reaches
-  // dep_read_target.  Every CTA counts its finished reads, and its finished scatter share
-  // when the call scatters.  Null: wait for the previous
-  // grid instead (griddepcontrol.wait).
+  // previous grid.  dep_scat counts CTAs of the layer's calls that finished their scatter
+  // share, dep_read CTAs that finished reading the buffer; both are counted in call order (a
+  // CTA counts once every CTA of the earlier calls has), so a count reaching the total of a
+  // prefix of the calls means exactly that prefix is done.  Waits (all >=):
+  //   hi rows:  *dep_scat >= dep_hi_target   (the scatters that wrote them)
+  //   lo rows:  *dep_scat >= dep_lo_target
+  //   scatter:  *dep_scat >= dep_scat_target (every earlier scatter) and
+  //             *dep_read >= dep_war_target  (every earlier call that read the rows it writes)
+  //   counting this CTA's reads: *dep_read >= dep_read_target (every earlier call) first.
+  // Null dep_scat: wait for the previous grid instead (griddepcontrol.wait).
   unsigned long long* dep_scat;
   unsigned long long* dep_read;
+  unsigned long long dep_hi_target;
+  unsigned long long dep_lo_target;
   unsigned long long dep_scat_target;
+  unsigned long long dep_war_target;
   unsigned long long dep_read_target;
 };
 

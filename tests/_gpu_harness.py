@@ -38,9 +38,20 @@ class Checker:
         assert absf <= MAX_ABS_FRAC, f"{what}: max-abs/max|V| {absf:.3e} > {MAX_ABS_FRAC}"
 
 
-def device_buffer_check(pat: pa.PatchAttention, layer: int, p: int, cur, prev, half=0):
+PIPEFUSION = (pa.PF_SCHED_PIPEFUSION, pa.PF_SCHED_PIPEFUSION_2H)
+
+
+def buffer_now(pat: pa.PatchAttention, layer: int):
+    """(K, V) of the layer's buffer as the next call sees it: the one half of the single-half
+    schedule, else the rows composed from both halves."""
+    if pat.cfg.schedule == pa.PF_SCHED_PIPEFUSION:
+        return pat.buffer_kv(layer, 0)
+    return pat.buffer_as_it_stands(layer)
+
+
+def device_buffer_check(pat: pa.PatchAttention, layer: int, p: int, cur, prev):
     """Bit-exact: buffer rows of patches <= p hold this step's K/V, the rest the previous step's."""
-    kb, vb = pat.buffer_kv(layer, half)
+    kb, vb = buffer_now(pat, layer)
     P = pat.plen
     hi = (p + 1) * P
     for buf, now, old in ((kb, cur["k"], prev["k"]), (vb, cur["v"], prev["v"])):
@@ -48,8 +59,8 @@ def device_buffer_check(pat: pa.PatchAttention, layer: int, p: int, cur, prev, h
         assert torch.equal(buf[:, hi:].view(torch.int16), old[:, hi:].view(torch.int16)), "stale rows"
 
 
-def oracle_buffer_check(pat: pa.PatchAttention, layer: int, p: int, cur, prev, half=0):
-    kb, vb = pat.buffer_kv(layer, half)
+def oracle_buffer_check(pat: pa.PatchAttention, layer: int, p: int, cur, prev):
+    kb, vb = buffer_now(pat, layer)
     for buf, now, old in ((kb, cur["k"], prev["k"]), (vb, cur["v"], prev["v"])):
         got = buf.cpu().view(torch.int16).numpy()[0]
         exp = oracle.expected_buffer(now.cpu().view(torch.int16).numpy()[0],
@@ -115,7 +126,7 @@ def run_workload(wl: synth.AttnWorkload, steps: Optional[int] = None, full_check
                     k_p = cur["k"][:, sl].contiguous()
                     v_p = cur["v"][:, sl].contiguous()
                     o = pat.step(layer, p, q_p, k_p, v_p, cur["k_txt"], cur["v_txt"])
-                    if schedule == pa.PF_SCHED_PIPEFUSION:
+                    if schedule in PIPEFUSION:
                         device_buffer_check(pat, layer, p, cur, pv)
                         if oracle_buffer(s, layer, p):
                             oracle_buffer_check(pat, layer, p, cur, pv)
@@ -148,7 +159,7 @@ def run_workload(wl: synth.AttnWorkload, steps: Optional[int] = None, full_check
 
 
 def _ref(wl, cur_cpu, prev_cpu, p, b, rows, heads, schedule):
-    if schedule == pa.PF_SCHED_PIPEFUSION:
+    if schedule in PIPEFUSION:
         return oracle_patch_output(wl, cur_cpu, prev_cpu, p, b, rows, heads)
     sl = slice(None) if heads is None else heads
     take = lambda t: f64(t[b][:, sl])
@@ -159,7 +170,7 @@ def _ref(wl, cur_cpu, prev_cpu, p, b, rows, heads, schedule):
 
 
 def _vmax(cur_cpu, prev_cpu, p, M, b, heads, schedule):
-    if schedule == pa.PF_SCHED_PIPEFUSION:
+    if schedule in PIPEFUSION:
         return vmax_used(cur_cpu, prev_cpu, p, M, b, heads)
     sl = slice(None) if heads is None else heads
     return max(float(cur_cpu["v"][b, :, sl].abs().max()), float(prev_cpu["v"][b, :, sl].abs().max()),

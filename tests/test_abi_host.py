@@ -195,6 +195,31 @@ def test_workspace_covers_the_text_query_call():
     assert pa.pf_workspace_bytes(many) >= 16 * 2 * 2 * 4 + 16
 
 
+def test_two_half_pipefusion_schedule_on_the_host():
+    # the same rows as PIPEFUSION in twice the buffer memory; order enforced the same way;
+    # only a step start can be restored; the half read starts at 0
+    one = _cfg(n_layers=2)
+    two = _cfg(n_layers=2, schedule=pa.PF_SCHED_PIPEFUSION_2H)
+    assert pa.pf_kvbuf_bytes(two) == 2 * pa.pf_kvbuf_bytes(one)
+    assert pa.pf_kvbuf_bytes(_cfg(schedule=3)) == 0
+    ctx = pa.pf_create(two, [FAKE, FAKE])
+    try:
+        assert pa.pf_get_read_half(ctx, 0) == 0 and pa.pf_get_read_half(ctx, 1) == 0
+        with pytest.raises(pa.PatchAttnError) as e:
+            pa.pf_get_read_half(ctx, 2)
+        assert e.value.status == pa.PF_ERR_INVALID_ARG
+        with pytest.raises(pa.PatchAttnError) as e:
+            pa.pf_set_state(ctx, 0, 1)
+        assert e.value.status == pa.PF_ERR_UNSUPPORTED
+        pa.pf_set_state(ctx, 0, 0)
+        assert pa.pf_get_state(ctx, 0) == 0
+        L = pa._lib()
+        # patch 1 before patch 0 is out of order (checked before anything is enqueued)
+        assert L.pf_patch_attn_step(ctx, 0, 1, FAKE, FAKE, FAKE, None, None, FAKE, None) == pa.PF_ERR_ORDER
+    finally:
+        pa.pf_destroy(ctx)
+
+
 def test_selftest_rejects_limits_out_of_range():
     L = pa._lib()
     assert L.pf_selftest_bounded_wait(0, None) == pa.PF_ERR_INVALID_ARG

@@ -24,50 +24,58 @@ def _wl(base, **kw):
     return dataclasses.replace(base, **kw)
 
 
-def test_tiny_every_call():
-    chk = run_workload(W["tiny"], full_check=lambda s, l, p: True, oracle_buffer=lambda s, l, p: True)
+PF, PF2 = pa.PF_SCHED_PIPEFUSION, pa.PF_SCHED_PIPEFUSION_2H
+
+
+@pytest.mark.parametrize("schedule", [PF, PF2])
+def test_tiny_every_call(schedule):
+    chk = run_workload(W["tiny"], full_check=lambda s, l, p: True, oracle_buffer=lambda s, l, p: True,
+                       schedule=schedule)
     assert chk.n == 3 * 4
 
 
-def test_pixart_all_steps():
+@pytest.mark.parametrize("schedule", [PF, PF2])
+def test_pixart_all_steps(schedule):
     wl = W["pixart"]
     last = wl.n_steps - 1
     chk = run_workload(wl, full_check=lambda s, l, p: s in (0, 1, 2, last),
                        sample_check=lambda s, l, p: True, n_sample_rows=32,
-                       oracle_buffer=lambda s, l, p: s in (1, last))
+                       oracle_buffer=lambda s, l, p: s in (1, last), schedule=schedule)
     assert chk.n > 0
 
 
-def test_sd3_full_size_sampled():
+@pytest.mark.parametrize("schedule", [PF, PF2])
+def test_sd3_full_size_sampled(schedule):
     wl = W["sd3"]
     S = wl.n_steps
-    chk = run_workload(wl, steps=S,
+    chk = run_workload(wl, steps=S, schedule=schedule,
                        full_check=lambda s, l, p: False,
                        sample_check=lambda s, l, p: (s in (0, 1, S - 1) and l in (0, 3)) or (s == 7 and p == 3),
                        n_sample_rows=8, oracle_buffer=lambda s, l, p: s == 1 and l == 0 and p in (0, 7))
     assert chk.n > 0
 
 
-def test_flux_full_size_sampled():
+@pytest.mark.parametrize("schedule", [PF, PF2])
+def test_flux_full_size_sampled(schedule):
     wl = W["flux"]
     S = wl.n_steps
     M = wl.n_patches
-    chk = run_workload(wl, steps=S,
+    chk = run_workload(wl, steps=S, schedule=schedule,
                        full_check=lambda s, l, p: False,
                        sample_check=lambda s, l, p: s in (0, 1, S - 1) and l in (0, 3) and p in (0, M // 2, M - 1),
                        n_sample_rows=4, oracle_buffer=lambda s, l, p: s == 1 and l == 3 and p == M - 1)
     assert chk.n > 0
 
 
-@pytest.mark.parametrize("split", [True, False])
+@pytest.mark.parametrize("split,schedule", [(True, PF), (False, PF), (True, PF2)])
 @pytest.mark.parametrize("d", [64, 72, 128])
-def test_ragged_shapes(d, split):
+def test_ragged_shapes(d, split, schedule):
     # patches that are not multiples of the 128-row tile, a ragged text tail, batch 2;
-    # with and without the key-range split across CTAs
+    # with and without the key-range split across CTAs; one buffer half or two
     wl = synth.AttnWorkload("ragged", batch=2, heads=3, head_dim=d, grid_h=20, grid_w=30,
                             n_patches=3, n_txt=77, n_layers=2, n_steps=3, ar_a=0.95, ar_b=0.3)
     chk = run_workload(wl, full_check=lambda s, l, p: True, oracle_buffer=lambda s, l, p: True,
-                       split=split)
+                       split=split, schedule=schedule)
     assert chk.n == 3 * 2 * 3 * 2
 
 

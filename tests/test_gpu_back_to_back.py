@@ -2,8 +2,10 @@
 
 Consecutive attention launches overlap on the GPU: a launch's CTAs may start while earlier
 micro-steps finish, and calls on the same layer buffer are ordered only by per-layer counters
-in the workspace (a call reads the buffer once the earlier calls on the layer have scattered
-into it, and scatters once they have finished reading it).  The other parity tests synchronise
+in the workspace (a call reads buffer rows once the earlier calls that wrote them have
+scattered, and scatters once the earlier calls that read the rows it overwrites have finished
+reading: with one buffer half every earlier call, with two the calls up to the previous
+step's call for the same patch).  The other parity tests synchronise
 after every call to check the buffer; here every call of a few diffusion steps -- the patch
 calls of every layer, then text-token queries on every layer at the end of each step -- is
 enqueued first, each into its own output, and only then checked: sampled rows of every call
@@ -22,11 +24,12 @@ from tests._oracle_util import f64
 
 pytestmark = pytest.mark.gpu
 
-PF, DF = pa.PF_SCHED_PIPEFUSION, pa.PF_SCHED_DISTRIFUSION
+PF, DF, PF2 = pa.PF_SCHED_PIPEFUSION, pa.PF_SCHED_DISTRIFUSION, pa.PF_SCHED_PIPEFUSION_2H
 
 
 @pytest.mark.parametrize("d,schedule,B", [(64, PF, 1), (72, PF, 1), (128, PF, 1), (64, DF, 1), (128, DF, 1),
-                                          (72, PF, 2)])
+                                          (72, PF, 2), (64, PF2, 1), (72, PF2, 1), (128, PF2, 1),
+                                          (72, PF2, 2)])
 def test_overlapped_micro_steps_match_the_oracle(d, schedule, B):
     wl = synth.AttnWorkload("b2b", batch=B, heads=4, head_dim=d, grid_h=64, grid_w=64,
                             n_patches=8, n_txt=77, n_layers=2, n_steps=3, ar_a=0.95, ar_b=0.3)
@@ -56,7 +59,7 @@ def test_overlapped_micro_steps_match_the_oracle(d, schedule, B):
         torch.cuda.synchronize()
         pat.check()  # no bounded wait gave up
         rng = np.random.default_rng(3)
-        attention = oracle.patch_attention if schedule == PF else oracle.distrifusion_attention
+        attention = oracle.distrifusion_attention if schedule == DF else oracle.patch_attention
         for (s, l, p), o in outs.items():
             cur, prev = steps[s][l], steps[max(s - 1, 0)][l]
             rows = sorted(set([0, P - 1] + list(rng.integers(0, P, 6))))
@@ -80,16 +83,16 @@ def test_overlapped_micro_steps_match_the_oracle(d, schedule, B):
             rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
             assert rel <= 5e-3, (s, l, "text", rel)
         for l in range(L):
+            # after the step's last patch the half being read holds the step
             last_k, last_v = steps[-1][l]["k"].view(torch.int16), steps[-1][l]["v"].view(torch.int16)
-            halves = (0,) if schedule == PF else (0, 1)
-            assert any(torch.equal(pat.buffer_kv(l, hf)[0].view(torch.int16), last_k) and
-                       torch.equal(pat.buffer_kv(l, hf)[1].view(torch.int16), last_v) for hf in halves), l
+            kb, vb = pat.buffer_kv(l, pat.read_half(l))
+            assert torch.equal(kb.view(torch.int16), last_k) and torch.equal(vb.view(torch.int16), last_v), l
         # between launches every split counter (parts arrived, partials written: two per query
         # tile of every pair) is back at 0, the merger of each query tile resets them; the
-        # per-layer ordering counters that follow them count, for every CTA of every call, one
-        # finished read of the buffer, and for every CTA of a patch call one finished scatter:
-        # every word before them is zero, and they are one (scatter, read) pair of non-zero
-        # counts per layer with more reads than scatters (partial slots follow the region)
+        # per-layer ordering counters that follow them count, for every CTA of a patch call,
+        # one finished scatter, and for every CTA of every call one finished read of the
+        # buffer: every word before them is zero, and they are one (scatter, read) pair of
+        # non-zero counts per layer with more reads than scatters (partial slots follow)
         assert pat.workspace is not None
         words = pat.workspace[:4096].view(torch.int64)
         first = int(torch.nonzero(words).flatten()[0])

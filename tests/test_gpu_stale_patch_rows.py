@@ -7,6 +7,7 @@ rows are made non-finite just before the call, with a patch length (200) that is
 multiple of the 128-row context tile, so the last tile of the rows before the patch reaches
 into the patch's rows.  The oracle never uses them, so the output must stay finite and match
 it: a kernel that read them (even under a softmax weight of 0, as 0 * inf) would produce NaN.
+With two buffer halves the rows of patch p in both halves are made non-finite.
 """
 import numpy as np
 import pytest
@@ -19,9 +20,10 @@ from tests._oracle_util import f64
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("split", [True, False])
+@pytest.mark.parametrize("split,schedule", [(True, pa.PF_SCHED_PIPEFUSION), (False, pa.PF_SCHED_PIPEFUSION),
+                                            (True, pa.PF_SCHED_PIPEFUSION_2H)])
 @pytest.mark.parametrize("d", [64, 72, 128])
-def test_stale_rows_of_the_patch_are_never_read(d, split):
+def test_stale_rows_of_the_patch_are_never_read(d, split, schedule):
     B, H, N, M, T = 1, 2, 600, 3, 10
     P = N // M
     g = torch.Generator(device="cuda").manual_seed(11)
@@ -29,15 +31,20 @@ def test_stale_rows_of_the_patch_are_never_read(d, split):
     k0, v0 = mk(B, N, H, d), mk(B, N, H, d)               # step 0: the buffer's start
     q1, k1, v1 = mk(B, N, H, d), mk(B, N, H, d), mk(B, N, H, d)  # step 1
     kt, vt = mk(B, T, H, d), mk(B, T, H, d)
-    pat = pa.PatchAttention(B, H, d, N, M, T, 1, split=split)
+    pat = pa.PatchAttention(B, H, d, N, M, T, 1, split=split, schedule=schedule)
     prev_k, prev_v = f64(k0[0]), f64(v0[0])
     try:
         pat.init_layer(0, k0, v0)
-        kb, vb = pat.buffer_kv(0)
+        rd = pat.read_half(0)
+        kb, vb = pat.buffer_kv(0, rd)
+        two = schedule == pa.PF_SCHED_PIPEFUSION_2H
+        # with two halves the call writes into the other half; its rows of patch p are stale
+        # too (from the step before the previous one, here never written)
+        kw, vw = pat.buffer_kv(0, 1 - rd) if two else (kb, vb)
         for p in range(M):
             sl = slice(p * P, (p + 1) * P)
-            kb[:, sl] = float("inf")
-            vb[:, sl] = float("inf")
+            for t in (kb, vb, kw, vw):
+                t[:, sl] = float("inf")
             prev_k[sl] = np.inf
             prev_v[sl] = np.inf
             o = pat.step(0, p, q1[:, sl].contiguous(), k1[:, sl].contiguous(), v1[:, sl].contiguous(),
@@ -53,9 +60,10 @@ def test_stale_rows_of_the_patch_are_never_read(d, split):
             rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
             assert rel <= 5e-3, (p, rel)
             assert np.abs(got - ref).max() <= 2e-2 * vmax, p
-            # the call replaced the patch's rows with the fresh ones, bit for bit
-            assert torch.equal(kb[:, sl].view(torch.int16), k1[:, sl].view(torch.int16))
-            assert torch.equal(vb[:, sl].view(torch.int16), v1[:, sl].view(torch.int16))
+            # the call replaced the patch's rows with the fresh ones, bit for bit (in the half
+            # being written)
+            assert torch.equal(kw[:, sl].view(torch.int16), k1[:, sl].view(torch.int16))
+            assert torch.equal(vw[:, sl].view(torch.int16), v1[:, sl].view(torch.int16))
         pat.check()
     finally:
         pat.close()

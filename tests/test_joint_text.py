@@ -65,7 +65,8 @@ def test_host_argument_checks():
 @pytest.mark.gpu
 @pytest.mark.parametrize("d,T,B", [(64, 154, 1), (72, 120, 1), (128, 512, 1), (128, 40, 1),
                                    (64, 300, 1), (128, 154, 2)])
-@pytest.mark.parametrize("schedule", [pa.PF_SCHED_PIPEFUSION, pa.PF_SCHED_DISTRIFUSION])
+@pytest.mark.parametrize("schedule", [pa.PF_SCHED_PIPEFUSION, pa.PF_SCHED_DISTRIFUSION,
+                                      pa.PF_SCHED_PIPEFUSION_2H])
 def test_text_queries_against_buffer_and_text(d, T, B, schedule):
     wl = synth.AttnWorkload("txt", B, 3, d, 24, 32, 4, T, 1, 2, 0.95, 0.3)
     P = wl.patch_len
@@ -85,11 +86,11 @@ def test_text_queries_against_buffer_and_text(d, T, B, schedule):
                 pat.step(0, p, cur["q"][:, sl].contiguous(), cur["k"][:, sl].contiguous(),
                          cur["v"][:, sl].contiguous(), cur["k_txt"], cur["v_txt"])
                 if p == 1:
-                    # mid-step: the buffer holds this step for patches <= 1 under PipeFusion,
-                    # the previous step everywhere under DistriFusion
+                    # mid-step: the buffer holds this step for patches <= 1 under PipeFusion
+                    # (either layout), the previous step everywhere under DistriFusion
                     o = pat.text_step(0, q_txt, cur["k_txt"], cur["v_txt"])
                     for bi in range(B):
-                        if schedule == pa.PF_SCHED_PIPEFUSION:
+                        if schedule != pa.PF_SCHED_DISTRIFUSION:
                             kb = oracle.expected_buffer(f64(cur["k"][bi]), f64(prev["k"][bi]), 1, 4)
                             vb = oracle.expected_buffer(f64(cur["v"][bi]), f64(prev["v"][bi]), 1, 4)
                         else:
