@@ -128,6 +128,12 @@ pf_status pf_kvbuf_init(pf_ctx* ctx, int layer, const void* k_full, const void* 
  * them), under PF_SCHED_DISTRIFUSION and PF_SCHED_PIPEFUSION_2H into the other half, which
  * becomes the half read once all M patches of the step have been called (PIPEFUSION_2H reads
  * the rows of patches < p from that other half).  o_p must not alias any input.
+ * Overlap: the attention kernels are launched as programmatic dependents, so when the
+ * previous work on the stream is another attention call of this library, this call's grid
+ * may start before that one has finished.  It orders itself against it for the buffer, its
+ * output and the workspace, but reads its own inputs (q_p, k_p, v_p, k_txt, v_txt) at once:
+ * an input must not be the output of the attention call directly before it on the stream
+ * (any other kernel in between, or a synchronisation, orders them as usual).
  * Errors: PF_ERR_STATE before pf_kvbuf_init(layer); PF_ERR_ORDER if `patch` is not the
  * layer's next patch (PipeFusion) or was already called this step (DistriFusion);
  * PF_ERR_INVALID_ARG / PF_ERR_ALIGN for bad pointers. */
@@ -142,7 +148,9 @@ pf_status pf_patch_attn_step(pf_ctx* ctx, int layer, int patch, const void* q_p,
  * and the patch counter is not moved.  "As it stands": under PF_SCHED_PIPEFUSION_2H, the
  * rows of the step's patches called so far and the previous step's rows of the others;
  * under PF_SCHED_DISTRIFUSION, the half being read.
- *   q_txt, k_txt, v_txt, o_txt : [B, T, H, d] bf16 (o_txt must not alias an input)
+ *   q_txt, k_txt, v_txt, o_txt : [B, T, H, d] bf16 (o_txt must not alias an input; the
+ *   inputs must not be the output of the attention call directly before it on the stream,
+ *   as for pf_patch_attn_step)
  * Errors: PF_ERR_SHAPE if the configuration has no text tokens; PF_ERR_STATE before
  * pf_kvbuf_init(layer). */
 pf_status pf_text_attn_step(pf_ctx* ctx, int layer, const void* q_txt, const void* k_txt,

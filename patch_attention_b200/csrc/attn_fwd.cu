@@ -418,10 +418,11 @@ __device__ __forceinline__ void scatter_share(const AttnParams& p, int lane) {
   }
 }
 
-// The producer's wait before its first tile of buffer rows of one kind: hi rows (src 3) were
-// written by calls of earlier epochs, lo rows (src 1) by earlier calls that may belong to
-// this epoch.  Without counters, one wait for the previous grid covers both.  False when a
-// bounded wait gave up.
+// The producer's wait before its first tile of buffer rows of one kind: hi rows (src 3) and
+// lo rows (src 1) each have the scatter count the host gave for the calls that wrote them
+// (with two buffer halves the hi rows were written in earlier steps, the lo rows by the
+// step's earlier calls).  Without counters, one wait for the previous grid covers both.
+// False when a bounded wait gave up.
 __device__ __forceinline__ bool buffer_rows_ready(const AttnParams& p, int src, bool& hi_done,
                                                   bool& lo_done, const volatile int* abort) {
   if (p.dep_scat == nullptr) {
@@ -657,8 +658,8 @@ __global__ void __launch_bounds__(kHrThreads, 1) patch_attn_hr_kernel(const __gr
   seg.init(p);
   const int n_all = seg.total();
   // part r takes context tiles [ceil(r n / k), ceil((r + 1) n / k)): the first parts take the
-  // extra tiles, and part 0 starts with the fresh rows, which it may compute before the
-  // previous micro-step has finished with the buffer
+  // extra tiles; the walk starts with the call's own tensors (fresh rows, text), which need
+  // nothing from earlier micro-steps
   const int j0 = static_cast<int>((static_cast<long long>(part) * n_all + p.n_split - 1) / p.n_split);
   const int j1 = static_cast<int>((static_cast<long long>(part + 1) * n_all + p.n_split - 1) / p.n_split);
   const int n_tiles = j1 - j0;  // this CTA's context tiles: j0 .. j1-1
@@ -1250,8 +1251,8 @@ __global__ void __launch_bounds__(kThreads, 1) patch_attn_sn_kernel(const __grid
   seg.init(p);
   const int n_all = seg.total();
   // part r takes context tiles [ceil(r n / k), ceil((r + 1) n / k)): the first parts take the
-  // extra tiles, and part 0 starts with the fresh rows, which it may compute before the
-  // previous micro-step has finished with the buffer
+  // extra tiles; the walk starts with the call's own tensors (fresh rows, text), which need
+  // nothing from earlier micro-steps
   const int j0 = static_cast<int>((static_cast<long long>(part) * n_all + p.n_split - 1) / p.n_split);
   const int j1 = static_cast<int>((static_cast<long long>(part + 1) * n_all + p.n_split - 1) / p.n_split);
   const int n_tiles = j1 - j0;  // this CTA's context tiles: j0 .. j1-1
