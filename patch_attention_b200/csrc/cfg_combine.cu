@@ -47,6 +47,10 @@ __global__ void __launch_bounds__(kThreads) cfg_partial_kernel(
     float4* __restrict__ out_f32, uint2* __restrict__ out_bf16, double2* __restrict__ partials) {
   // let the finalize kernel be scheduled now; it waits for this grid's completion itself
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // launched as a programmatic dependent of the previous work on the stream (often the last
+  // attention launch of a step): wait until that grid has finished and its writes are
+  // visible before touching memory
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.y;
   const int g = blockIdx.x;
   const int G = gridDim.x;
@@ -116,6 +120,9 @@ __global__ void cfg_finalize_kernel(const double2* __restrict__ partials, int G,
   // launched as a programmatic dependent of cfg_partial_kernel: wait until that grid has
   // finished and its partials are visible
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the partial kernel is complete: the next work on the stream may be scheduled (it writes
+  // nothing this kernel reads before waiting for this grid itself)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int b = blockIdx.x;
   const int lane = threadIdx.x;
   double num = 0.0, den = 0.0;
@@ -197,22 +204,30 @@ cudaError_t launch_cfg_combine_relmae(const float* c, const float* u, int batch,
                                       void* workspace, cudaStream_t stream) {
   const int G = blocks_per_sample(batch, n);
   dim3 grid(G, batch);
-  cfg_partial_kernel<<<grid, kThreads, 0, stream>>>(
-      reinterpret_cast<const float4*>(c), reinterpret_cast<const float4*>(u), n / 4, w,
-      reinterpret_cast<float4*>(out_f32), reinterpret_cast<uint2*>(out_bf16),
-      reinterpret_cast<double2*>(workspace));
-  cudaError_t e = cudaGetLastError();
+  // both kernels are programmatic dependents: the partial kernel's launch overlaps the end of
+  // the previous grid (it waits for it with griddepcontrol.wait before touching memory), and
+  // the finalize is scheduled while the partial kernel runs (hiding its launch latency) and
+  // synchronises on it the same way
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t pcfg = {};
+  pcfg.gridDim = grid;
+  pcfg.blockDim = dim3(kThreads);
+  pcfg.dynamicSmemBytes = 0;
+  pcfg.stream = stream;
+  pcfg.attrs = attr;
+  pcfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&pcfg, cfg_partial_kernel, reinterpret_cast<const float4*>(c),
+                                     reinterpret_cast<const float4*>(u), n / 4, w,
+                                     reinterpret_cast<float4*>(out_f32), reinterpret_cast<uint2*>(out_bf16),
+                                     reinterpret_cast<double2*>(workspace));
   if (e != cudaSuccess) return e;
-  // programmatic dependent launch: the finalize is scheduled while the partial kernel runs
-  // (hiding its launch latency) and synchronises on it with griddepcontrol.wait
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(batch);
   cfg.blockDim = dim3(32);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, cfg_finalize_kernel, reinterpret_cast<const double2*>(workspace), G,

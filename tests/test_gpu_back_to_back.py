@@ -7,8 +7,8 @@ scattered, and scatters once the earlier calls that read the rows it overwrites 
 reading: with one buffer half every earlier call, with two the calls up to the previous
 step's call for the same patch).  The other parity tests synchronise
 after every call to check the buffer; here every call of a few diffusion steps -- the patch
-calls of every layer, then text-token queries on every layer at the end of each step -- is
-enqueued first, each into its own output, and only then checked: sampled rows of every call
+calls of every layer, text-token queries on every layer after patch 1 and again at the end of
+each step -- is enqueued first, each into its own output, and only then checked: sampled rows of every call
 against the fp64 oracle, the buffer against the last step, the device status word (a bounded
 wait that gave up would show as PF_ERR_TIMEOUT), the key-range split's counters, which must
 all be back at zero, and the per-layer ordering counters.
@@ -39,7 +39,7 @@ def test_overlapped_micro_steps_match_the_oracle(d, schedule, B):
     g = torch.Generator(device="cuda").manual_seed(5)
     q_txt = [torch.randn(B, T, wl.heads, d, device="cuda", generator=g).bfloat16() for _ in range(L)]
     pat = pa.PatchAttention(B, wl.heads, d, wl.n_img, M, T, L, schedule=schedule)
-    outs, txt_outs = {}, {}
+    outs, txt_outs, mid_outs = {}, {}, {}
     try:
         for l in range(L):
             pat.init_layer(l, steps[0][l]["k"], steps[0][l]["v"])
@@ -53,6 +53,11 @@ def test_overlapped_micro_steps_match_the_oracle(d, schedule, B):
                     q, k, v = patches[s][l][p]
                     t = steps[s][l]
                     outs[(s, l, p)] = pat.step(l, p, q, k, v, t["k_txt"], t["v_txt"])
+                if p == 1:
+                    # text queries in the middle of the step: the buffer as it stands
+                    for l in range(L):
+                        t = steps[s][l]
+                        mid_outs[(s, l)] = pat.text_step(l, q_txt[l], t["k_txt"], t["v_txt"])
             for l in range(L):
                 t = steps[s][l]
                 txt_outs[(s, l)] = pat.text_step(l, q_txt[l], t["k_txt"], t["v_txt"])
@@ -82,6 +87,24 @@ def test_overlapped_micro_steps_match_the_oracle(d, schedule, B):
             got = f64(o[bi][rows][:, h:h + 1])
             rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
             assert rel <= 5e-3, (s, l, "text", rel)
+        for (s, l), o in mid_outs.items():
+            # after patch 1: this step's rows for patches 0-1 and the previous step's for the
+            # rest under PipeFusion (either layout); the previous step everywhere under
+            # DistriFusion
+            cur, prev = steps[s][l], steps[max(s - 1, 0)][l]
+            h, bi = int(rng.integers(0, wl.heads)), int(rng.integers(0, B))
+            rows = sorted(set([0, T - 1] + list(rng.integers(0, T, 6))))
+            take = lambda x: f64(x[bi][:, h:h + 1])
+            if schedule == DF:
+                kb, vb = take(prev["k"]), take(prev["v"])
+            else:
+                kb = oracle.expected_buffer(take(cur["k"]), take(prev["k"]), 1, M)
+                vb = oracle.expected_buffer(take(cur["v"]), take(prev["v"]), 1, M)
+            ref = oracle.attend(take(q_txt[l])[rows], np.concatenate([kb, take(cur["k_txt"])]),
+                                np.concatenate([vb, take(cur["v_txt"])]), wl.softmax_scale)
+            got = f64(o[bi][rows][:, h:h + 1])
+            rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+            assert rel <= 5e-3, (s, l, "mid-step text", rel)
         for l in range(L):
             # after the step's last patch the half being read holds the step
             last_k, last_v = steps[-1][l]["k"].view(torch.int16), steps[-1][l]["v"].view(torch.int16)
