@@ -126,7 +126,8 @@ def test_overlapped_micro_steps_match_the_oracle(d, schedule, B):
         pat.close()
 
 
-def test_workspace_detached_and_attached_between_steps():
+@pytest.mark.parametrize("schedule", [PF, PF2])
+def test_workspace_detached_and_attached_between_steps(schedule):
     """Calls without a workspace wait for the previous grid; attaching a workspace again zeroes
     the counters (ordered after the calls still running on the stream) and restarts the host's
     targets.  Steps alternate between the two, still without host synchronisation."""
@@ -136,7 +137,7 @@ def test_workspace_detached_and_attached_between_steps():
     S, L, M, P = wl.n_steps, wl.n_layers, wl.n_patches, wl.patch_len
     gen = synth.AttnInputs(wl, seed=8, device="cuda")
     steps = [[gen.step_tensors(l) for l in range(L)] for _ in range(S)]
-    pat = pa.PatchAttention(1, wl.heads, d, wl.n_img, M, wl.n_txt, L)
+    pat = pa.PatchAttention(1, wl.heads, d, wl.n_img, M, wl.n_txt, L, schedule=schedule)
     ws = pat.workspace
     assert ws is not None
     outs = {}
@@ -166,7 +167,7 @@ def test_workspace_detached_and_attached_between_steps():
             rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
             assert rel <= 5e-3, (s, l, p, rel)
         for l in range(L):
-            kb, vb = pat.buffer_kv(l)
+            kb, vb = pat.buffer_kv(l, pat.read_half(l))
             assert torch.equal(kb.view(torch.int16), steps[-1][l]["k"].view(torch.int16))
             assert torch.equal(vb.view(torch.int16), steps[-1][l]["v"].view(torch.int16))
     finally:
