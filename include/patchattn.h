@@ -181,9 +181,9 @@ size_t pf_workspace_bytes(const pf_config* cfg);
 
 /* Attach a caller-owned device workspace (16-byte aligned, >= pf_workspace_bytes(cfg))
  * to ctx and zero its counters on `stream`.  ws = NULL detaches it (no key-range split).
- * Calls that share a workspace must not run concurrently (one workspace per stream), and the
- * calls of a context run on that one stream.  After PF_ERR_TIMEOUT, set the workspace again
- * to re-zero the counters. */
+ * A workspace belongs to one context (its ordering counters are counted against that
+ * context's host-side totals), and the calls of a context run on one stream.  After
+ * PF_ERR_TIMEOUT, set the workspace again to re-zero the counters. */
 pf_status pf_set_workspace(pf_ctx* ctx, void* ws, size_t ws_bytes, void* stream);
 
 /* Next patch index the layer expects (0 at the start of a step).  Checkpoint helper: a
