@@ -120,9 +120,6 @@ __global__ void cfg_finalize_kernel(const double2* __restrict__ partials, int G,
   // launched as a programmatic dependent of cfg_partial_kernel: wait until that grid has
   // finished and its partials are visible
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  // the partial kernel is complete: the next work on the stream may be scheduled (it writes
-  // nothing this kernel reads before waiting for this grid itself)
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int b = blockIdx.x;
   const int lane = threadIdx.x;
   double num = 0.0, den = 0.0;
